@@ -1,0 +1,547 @@
+// bf16 eviction-masked attention backward on sm_100a tensor cores.
+//
+// Textbook softmax-attention gradients restricted to the visible pairs of the
+// replayed trace ("KV-streams: speeding up agentic RL by operating on the KV
+// cache directly", trainer replay; "KV-streams for Efficient Compaction in
+// Agentic Reinforcement Learning", Fig. 2(A)):
+//   P = exp(S - LSE), dV = P^T dO, dP = dO V^T, dS = P (dP - D),
+//   dQ = scale dS K, dK = scale dS^T Q, D = rowsum(dO * O).
+//
+// Three launches, no atomics (deterministic):
+//   prep   D and LSE*log2(e) per (trace, head, row), padded to whole tiles
+//   dK/dV  one CTA per (key tile, kv head, trace); walks the column lists of
+//          the mask for every query head of the group. Transposed products
+//          S^T = K Q^T and dP^T = V dO^T put one key per TMEM lane, so P^T and
+//          dS^T are written back to TMEM in bf16 and used as the A operand of
+//          dV += P^T dO and dK += dS^T Q. Within a tile a key's visible query
+//          rows form one interval (j <= t < kappa_j), so masking needs only
+//          kappa_j, not the bit rows.
+//   dQ     one CTA per (query tile, head, trace) over the row lists:
+//          S = Q K^T, dP = dO V^T, dS (bit-masked) to TMEM, dQ += dS K.
+// Warp roles as in the forward: warp 0 TMA, warp 1 TMEM + MMA issue, warps
+// 2..5 elementwise (thread = TMEM lane).
+#include "common.cuh"
+
+namespace kvs {
+
+bool make_tmap_bnhd(CUtensorMap *map, const void *base, int B, int N, int H);
+
+constexpr int kBwdThreads = 192;
+constexpr uint32_t kTile = 128 * 128 * 2;
+
+__device__ __forceinline__ bool wait_done(uint64_t *bar, uint32_t parity) {
+    uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(bar, parity))
+        if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+    return true;
+}
+
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
+                                          int32_t *status) {
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, status));
+}
+
+// D[b][h][t] = <dO, O>, L2[b][h][t] = lse * log2(e); rows t >= N get 0. Tpad = T*128.
+__global__ void k_bwd_prep(const __nv_bfloat16 *__restrict__ o, const __nv_bfloat16 *__restrict__ dO,
+                           const float *__restrict__ lse, int32_t B, int32_t N, int32_t Hq,
+                           int32_t Tpad, float *__restrict__ Drow, float *__restrict__ L2) {
+    const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= (int64_t)B * Hq * Tpad) return;
+    const int64_t t = row % Tpad, bh = row / Tpad, h = bh % Hq, b = bh / Hq;
+    float s = 0.f, l2 = 0.f;
+    if (t < N) {
+        const int64_t off = ((b * N + t) * Hq + h) * 128 + lane * 4;
+        const uint2 a = *reinterpret_cast<const uint2 *>(o + off);
+        const uint2 c = *reinterpret_cast<const uint2 *>(dO + off);
+        s = bf16_lo(a.x) * bf16_lo(c.x) + bf16_hi(a.x) * bf16_hi(c.x) + bf16_lo(a.y) * bf16_lo(c.y) +
+            bf16_hi(a.y) * bf16_hi(c.y);
+        for (int k = 16; k; k >>= 1) s += __shfl_xor_sync(0xffffffffu, s, k);
+        l2 = lse[(b * Hq + h) * N + t] * 1.4426950408889634f;
+    }
+    if (lane == 0) {
+        Drow[row] = s;
+        L2[row] = l2;
+    }
+}
+
+// ---------------------------------------------------------------------- dK / dV
+
+struct DkvSmem {
+    uint8_t k[kTile];
+    uint8_t v[kTile];
+    uint8_t q[2][kTile];
+    uint8_t dout[2][kTile];
+    float l2[2][128];
+    float dd[2][128];
+    uint64_t kv_full, full[2], empty[2], st_full, dp_full, p_ready, ds_ready, acc_done, fin;
+    uint32_t tmem_base;
+    int abort;
+};
+
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    k_attn_dkdv_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                   kvs_tile_mask m, int32_t Hq, int32_t Hkv, float scale, float scale_log2,
+                   const float *__restrict__ Drow, const float *__restrict__ L2,
+                   __nv_bfloat16 *__restrict__ dk, __nv_bfloat16 *__restrict__ dv, int32_t *status) {
+    extern __shared__ uint8_t smem_raw[];
+    DkvSmem &S = *reinterpret_cast<DkvSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int B = m.B, N = m.N, T = m.T, G = Hq / Hkv, Tpad = T * 128;
+    // key tiles with the longest column lists (small kj) first
+    const int64_t idx = blockIdx.x;
+    const int kj = (int)(idx / ((int64_t)B * Hkv));
+    const int rem = (int)(idx % ((int64_t)B * Hkv));
+    const int kvh = rem % Hkv, b = rem / Hkv;
+    const int k0 = kj * 128;
+    const int32_t c0 = m.col_ptr[b * T + kj], ncol = m.col_ptr[b * T + kj + 1] - c0;
+    const int nw = ncol * G;
+    if (grid_timed_out(status)) return;
+
+    if (threadIdx.x == 0) {
+        mbar_init(&S.kv_full, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&S.full[i], 1);
+            mbar_init(&S.empty[i], 1);
+        }
+        mbar_init(&S.st_full, 1);
+        mbar_init(&S.dp_full, 1);
+        mbar_init(&S.p_ready, 128);
+        mbar_init(&S.ds_ready, 128);
+        mbar_init(&S.acc_done, 1);
+        mbar_init(&S.fin, 1);
+        S.abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(&S.tmem_base, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = S.tmem_base;
+    volatile int *abort = &S.abort;
+    constexpr uint32_t cST = 0, cDP = 128, cDV = 256, cDK = 384;
+
+    if (warp == 0) {
+        if (lane == 0 && nw > 0) {
+            mbar_expect_tx(&S.kv_full, 2 * kTile);
+            tma_load_4d(S.k, &tmK, &S.kv_full, 0, kvh, k0, b);
+            tma_load_4d(S.k + kTile / 2, &tmK, &S.kv_full, 64, kvh, k0, b);
+            tma_load_4d(S.v, &tmV, &S.kv_full, 0, kvh, k0, b);
+            tma_load_4d(S.v + kTile / 2, &tmV, &S.kv_full, 64, kvh, k0, b);
+            for (int n = 0; n < nw; ++n) {
+                const int s = n & 1;
+                if (n >= 2 && !mbar_wait(&S.empty[s], ((n >> 1) - 1) & 1, abort, status)) break;
+                const int e = n / G, g = n % G, h = kvh * G + g;
+                const int q0 = m.col_row[c0 + e] * 128;
+                mbar_expect_tx(&S.full[s], 2 * kTile + 1024);
+                tma_load_4d(S.q[s], &tmQ, &S.full[s], 0, h, q0, b);
+                tma_load_4d(S.q[s] + kTile / 2, &tmQ, &S.full[s], 64, h, q0, b);
+                tma_load_4d(S.dout[s], &tmO, &S.full[s], 0, h, q0, b);
+                tma_load_4d(S.dout[s] + kTile / 2, &tmO, &S.full[s], 64, h, q0, b);
+                const int64_t ro = ((int64_t)b * Hq + h) * Tpad + q0;
+                bulk_load(S.l2[s], L2 + ro, 512, &S.full[s]);
+                bulk_load(S.dd[s], Drow + ro, 512, &S.full[s]);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && nw > 0) {
+            const uint32_t idKM = idesc_bf16(128, 128, false, false);  // both K-major
+            const uint32_t idMN = idesc_bf16(128, 128, false, true);   // B MN-major
+            const uint32_t ka = smem_u32(S.k), va = smem_u32(S.v);
+            bool ok = mbar_wait(&S.kv_full, 0, abort, status);
+            for (int n = 0; ok && n < nw; ++n) {
+                const int s = n & 1;
+                if (!mbar_wait(&S.full[s], (n >> 1) & 1, abort, status)) break;
+                tc_fence_after();
+                const uint32_t qa = smem_u32(S.q[s]), oa = smem_u32(S.dout[s]);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t off = (kk >> 2) * (kTile / 2) + (kk & 3) * 32;
+                    mma_ss(tmem + cST, sw128_desc(ka + off, 16, 1024), sw128_desc(qa + off, 16, 1024),
+                           idKM, kk > 0);
+                }
+                mma_commit(&S.st_full);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t off = (kk >> 2) * (kTile / 2) + (kk & 3) * 32;
+                    mma_ss(tmem + cDP, sw128_desc(va + off, 16, 1024), sw128_desc(oa + off, 16, 1024),
+                           idKM, kk > 0);
+                }
+                mma_commit(&S.dp_full);
+                if (!mbar_wait(&S.p_ready, n & 1, abort, status)) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_ts(tmem + cDV, tmem + cST + kk * 8, sw128_desc(oa + kk * 2048, kTile / 2, 1024),
+                           idMN, (n > 0 || kk > 0) ? 1u : 0u);
+                if (!mbar_wait(&S.ds_ready, n & 1, abort, status)) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_ts(tmem + cDK, tmem + cDP + kk * 8, sw128_desc(qa + kk * 2048, kTile / 2, 1024),
+                           idMN, (n > 0 || kk > 0) ? 1u : 0u);
+                mma_commit(&S.empty[s]);
+            }
+            mma_commit(&S.acc_done);
+            mma_commit(&S.fin);
+            wait_done(&S.fin, 0);
+        }
+    } else {
+        const int quad = warp & 3;
+        const int c = quad * 32 + lane;  // key row within the tile
+        const int j = k0 + c;
+        const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+        const int32_t kap = j < N ? m.kappa[(int64_t)b * N + j] : 0;
+        bool ok = true;
+        for (int n = 0; n < nw; ++n) {
+            const int s = n & 1;
+            const int e = n / G;
+            const int q0 = m.col_row[c0 + e] * 128;
+            const bool full = m.col_pidx[c0 + e] < 0;
+            int rlo = 0, rhi = 128;
+            if (!full) {
+                if (j >= N) {
+                    rlo = rhi = 0;
+                } else {
+                    const int64_t lo = (int64_t)j - q0, hi = (int64_t)(kap < N ? kap : N) - q0;
+                    rlo = (int)(lo < 0 ? 0 : (lo > 128 ? 128 : lo));
+                    rhi = (int)(hi < 0 ? 0 : (hi > 128 ? 128 : hi));
+                }
+            }
+            if (!warp_wait(&S.full[s], (n >> 1) & 1, abort, status) ||
+                !warp_wait(&S.st_full, n & 1, abort, status)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            float p[128];
+            {
+                uint32_t r[4][32];
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc) tmem_ld32(tmem + lane_off + cST + cc * 32, r[cc]);
+                tmem_ld_wait();
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc)
+#pragma unroll
+                    for (int jj = 0; jj < 32; ++jj) {
+                        const int rr = cc * 32 + jj;
+                        const float x = __uint_as_float(r[cc][jj]) * scale_log2 - S.l2[s][rr];
+                        p[rr] = (rr >= rlo && rr < rhi) ? ex2(x) : 0.f;
+                    }
+            }
+            {
+                uint32_t pk[2][32];
+#pragma unroll
+                for (int rr = 0; rr < 128; rr += 2) pk[rr >> 6][(rr & 63) >> 1] = pack_bf16(p[rr], p[rr + 1]);
+                tmem_st32(tmem + lane_off + cST, pk[0]);
+                tmem_st32(tmem + lane_off + cST + 32, pk[1]);
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(&S.p_ready);
+            if (!warp_wait(&S.dp_full, n & 1, abort, status)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                uint32_t pk[32];
+#pragma unroll
+                for (int cc = 0; cc < 2; ++cc) {
+                    uint32_t r[32];
+                    tmem_ld32(tmem + lane_off + cDP + (half * 2 + cc) * 32, r);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int jj = 0; jj < 32; jj += 2) {
+                        const int rr = (half * 2 + cc) * 32 + jj;
+                        const float d0 = p[rr] * (__uint_as_float(r[jj]) - S.dd[s][rr]);
+                        const float d1 = p[rr + 1] * (__uint_as_float(r[jj + 1]) - S.dd[s][rr + 1]);
+                        pk[cc * 16 + (jj >> 1)] = pack_bf16(d0, d1);
+                    }
+                }
+                tmem_st32(tmem + lane_off + cDP + half * 32, pk);
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(&S.ds_ready);
+        }
+        if (ok && nw > 0 && warp_wait(&S.acc_done, 0, abort, status)) {
+            tc_fence_after();
+            const int64_t ro = (((int64_t)b * N + j) * Hkv + kvh) * 128;
+#pragma unroll
+            for (int which = 0; which < 2; ++which) {
+                __nv_bfloat16 *dst = (which ? dk : dv) + ro;
+                const float f = which ? scale : 1.f;
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc) {
+                    uint32_t r[32];
+                    tmem_ld32(tmem + lane_off + (which ? cDK : cDV) + cc * 32, r);
+                    tmem_ld_wait();
+                    if (j < N) {
+#pragma unroll
+                        for (int jj = 0; jj < 32; jj += 8) {
+                            uint4 w;
+                            w.x = pack_bf16(__uint_as_float(r[jj]) * f, __uint_as_float(r[jj + 1]) * f);
+                            w.y = pack_bf16(__uint_as_float(r[jj + 2]) * f, __uint_as_float(r[jj + 3]) * f);
+                            w.z = pack_bf16(__uint_as_float(r[jj + 4]) * f, __uint_as_float(r[jj + 5]) * f);
+                            w.w = pack_bf16(__uint_as_float(r[jj + 6]) * f, __uint_as_float(r[jj + 7]) * f);
+                            *reinterpret_cast<uint4 *>(dst + cc * 32 + jj) = w;
+                        }
+                    }
+                }
+            }
+        } else if (nw == 0 && j < N) {
+            // a key no query sees (cannot happen for a valid mask: the diagonal is visible)
+            const int64_t ro = (((int64_t)b * N + j) * Hkv + kvh) * 128;
+            for (int i = 0; i < 128; i += 8) {
+                *reinterpret_cast<uint4 *>(dk + ro + i) = make_uint4(0, 0, 0, 0);
+                *reinterpret_cast<uint4 *>(dv + ro + i) = make_uint4(0, 0, 0, 0);
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+// ---------------------------------------------------------------------- dQ
+
+struct DqSmem {
+    uint8_t q[kTile];
+    uint8_t dout[kTile];
+    uint8_t k[2][kTile];
+    uint8_t v[2][kTile];
+    uint64_t qo_full, full[2], empty[2], s_full, dp_full, ds_ready, acc_done, fin;
+    uint32_t tmem_base;
+    int abort;
+};
+
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    k_attn_dq_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                 kvs_tile_mask m, int32_t Hq, int32_t Hkv, float scale, float scale_log2,
+                 const float *__restrict__ Drow, const float *__restrict__ L2,
+                 __nv_bfloat16 *__restrict__ dq, int32_t *status) {
+    extern __shared__ uint8_t smem_raw[];
+    DqSmem &S = *reinterpret_cast<DqSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                           ~uintptr_t(1023));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int B = m.B, N = m.N, T = m.T, G = Hq / Hkv, Tpad = T * 128;
+    const int64_t idx = blockIdx.x;
+    const int qi = T - 1 - (int)(idx / ((int64_t)B * Hq));
+    const int rem = (int)(idx % ((int64_t)B * Hq));
+    const int hq = rem % Hq, b = rem / Hq, kvh = hq / G;
+    const int q0 = qi * 128;
+    const int32_t e0 = m.row_ptr[b * T + qi], nt = m.row_ptr[b * T + qi + 1] - e0;
+    if (grid_timed_out(status)) return;
+
+    if (threadIdx.x == 0) {
+        mbar_init(&S.qo_full, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&S.full[i], 1);
+            mbar_init(&S.empty[i], 1);
+        }
+        mbar_init(&S.s_full, 1);
+        mbar_init(&S.dp_full, 1);
+        mbar_init(&S.ds_ready, 128);
+        mbar_init(&S.acc_done, 1);
+        mbar_init(&S.fin, 1);
+        S.abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(&S.tmem_base, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = S.tmem_base;
+    volatile int *abort = &S.abort;
+    constexpr uint32_t cS = 0, cDP = 128, cDQ = 256;
+
+    if (warp == 0) {
+        if (lane == 0 && nt > 0) {
+            mbar_expect_tx(&S.qo_full, 2 * kTile);
+            tma_load_4d(S.q, &tmQ, &S.qo_full, 0, hq, q0, b);
+            tma_load_4d(S.q + kTile / 2, &tmQ, &S.qo_full, 64, hq, q0, b);
+            tma_load_4d(S.dout, &tmO, &S.qo_full, 0, hq, q0, b);
+            tma_load_4d(S.dout + kTile / 2, &tmO, &S.qo_full, 64, hq, q0, b);
+            for (int n = 0; n < nt; ++n) {
+                const int s = n & 1;
+                if (n >= 2 && !mbar_wait(&S.empty[s], ((n >> 1) - 1) & 1, abort, status)) break;
+                const int k0 = m.row_col[e0 + n] * 128;
+                mbar_expect_tx(&S.full[s], 2 * kTile);
+                tma_load_4d(S.k[s], &tmK, &S.full[s], 0, kvh, k0, b);
+                tma_load_4d(S.k[s] + kTile / 2, &tmK, &S.full[s], 64, kvh, k0, b);
+                tma_load_4d(S.v[s], &tmV, &S.full[s], 0, kvh, k0, b);
+                tma_load_4d(S.v[s] + kTile / 2, &tmV, &S.full[s], 64, kvh, k0, b);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && nt > 0) {
+            const uint32_t idKM = idesc_bf16(128, 128, false, false);
+            const uint32_t idMN = idesc_bf16(128, 128, false, true);
+            const uint32_t qa = smem_u32(S.q), oa = smem_u32(S.dout);
+            bool ok = mbar_wait(&S.qo_full, 0, abort, status);
+            for (int n = 0; ok && n < nt; ++n) {
+                const int s = n & 1;
+                if (!mbar_wait(&S.full[s], (n >> 1) & 1, abort, status)) break;
+                tc_fence_after();
+                const uint32_t ka = smem_u32(S.k[s]), va = smem_u32(S.v[s]);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t off = (kk >> 2) * (kTile / 2) + (kk & 3) * 32;
+                    mma_ss(tmem + cS, sw128_desc(qa + off, 16, 1024), sw128_desc(ka + off, 16, 1024),
+                           idKM, kk > 0);
+                }
+                mma_commit(&S.s_full);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t off = (kk >> 2) * (kTile / 2) + (kk & 3) * 32;
+                    mma_ss(tmem + cDP, sw128_desc(oa + off, 16, 1024), sw128_desc(va + off, 16, 1024),
+                           idKM, kk > 0);
+                }
+                mma_commit(&S.dp_full);
+                if (!mbar_wait(&S.ds_ready, n & 1, abort, status)) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_ts(tmem + cDQ, tmem + cS + kk * 8, sw128_desc(ka + kk * 2048, kTile / 2, 1024),
+                           idMN, (n > 0 || kk > 0) ? 1u : 0u);
+                mma_commit(&S.empty[s]);
+            }
+            mma_commit(&S.acc_done);
+            mma_commit(&S.fin);
+            wait_done(&S.fin, 0);
+        }
+    } else {
+        const int quad = warp & 3;
+        const int row = quad * 32 + lane;
+        const int t = q0 + row;
+        const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+        const int64_t ro = ((int64_t)b * Hq + hq) * Tpad + t;
+        const float l2 = L2[ro], dd = Drow[ro];
+        bool ok = true;
+        for (int n = 0; n < nt; ++n) {
+            const int32_t pid = m.row_pidx[e0 + n];
+            uint4 bits = make_uint4(~0u, ~0u, ~0u, ~0u);
+            if (pid >= 0)
+                bits = *reinterpret_cast<const uint4 *>(m.bits + (int64_t)pid * 512 + row * 4);
+            const uint32_t wb[4] = {bits.x, bits.y, bits.z, bits.w};
+            if (!warp_wait(&S.s_full, n & 1, abort, status)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            float p[128];
+            {
+                uint32_t r[4][32];
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc) tmem_ld32(tmem + lane_off + cS + cc * 32, r[cc]);
+                tmem_ld_wait();
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc)
+#pragma unroll
+                    for (int jj = 0; jj < 32; ++jj)
+                        p[cc * 32 + jj] = ((wb[cc] >> jj) & 1u)
+                                              ? ex2(__uint_as_float(r[cc][jj]) * scale_log2 - l2)
+                                              : 0.f;
+            }
+            if (!warp_wait(&S.dp_full, n & 1, abort, status)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                uint32_t pk[32];
+#pragma unroll
+                for (int cc = 0; cc < 2; ++cc) {
+                    uint32_t r[32];
+                    tmem_ld32(tmem + lane_off + cDP + (half * 2 + cc) * 32, r);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int jj = 0; jj < 32; jj += 2) {
+                        const int kc = (half * 2 + cc) * 32 + jj;
+                        pk[cc * 16 + (jj >> 1)] = pack_bf16(p[kc] * (__uint_as_float(r[jj]) - dd),
+                                                            p[kc + 1] * (__uint_as_float(r[jj + 1]) - dd));
+                    }
+                }
+                tmem_st32(tmem + lane_off + cS + half * 32, pk);
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(&S.ds_ready);
+        }
+        if (ok && nt > 0 && warp_wait(&S.acc_done, 0, abort, status)) {
+            tc_fence_after();
+            __nv_bfloat16 *dst = dq + (((int64_t)b * N + t) * Hq + hq) * 128;
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+                uint32_t r[32];
+                tmem_ld32(tmem + lane_off + cDQ + cc * 32, r);
+                tmem_ld_wait();
+                if (t < N) {
+#pragma unroll
+                    for (int jj = 0; jj < 32; jj += 8) {
+                        uint4 w;
+                        w.x = pack_bf16(__uint_as_float(r[jj]) * scale, __uint_as_float(r[jj + 1]) * scale);
+                        w.y = pack_bf16(__uint_as_float(r[jj + 2]) * scale, __uint_as_float(r[jj + 3]) * scale);
+                        w.z = pack_bf16(__uint_as_float(r[jj + 4]) * scale, __uint_as_float(r[jj + 5]) * scale);
+                        w.w = pack_bf16(__uint_as_float(r[jj + 6]) * scale, __uint_as_float(r[jj + 7]) * scale);
+                        *reinterpret_cast<uint4 *>(dst + cc * 32 + jj) = w;
+                    }
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+size_t bwd_tc_ws_bytes(int32_t B, int32_t N, int32_t Hq) {
+    const int64_t Tpad = (int64_t)((N + 127) / 128) * 128;
+    return 2 * (size_t)B * Hq * Tpad * sizeof(float);
+}
+
+cudaError_t launch_bwd_tc(const void *q, const void *k, const void *v, const void *o,
+                          const void *dO, const float *lse, const kvs_tile_mask &m, int32_t Hq,
+                          int32_t Hkv, float scale, void *dq, void *dk, void *dv, void *ws,
+                          int32_t *status, cudaStream_t s, bool *map_ok) {
+    CUtensorMap tq, tk, tv, to;
+    *map_ok = make_tmap_bnhd(&tq, q, m.B, m.N, Hq) && make_tmap_bnhd(&tk, k, m.B, m.N, Hkv) &&
+              make_tmap_bnhd(&tv, v, m.B, m.N, Hkv) && make_tmap_bnhd(&to, dO, m.B, m.N, Hq);
+    if (!*map_ok) return cudaSuccess;
+    const int32_t Tpad = m.T * 128;
+    float *Drow = (float *)ws;
+    float *L2 = Drow + (size_t)m.B * Hq * Tpad;
+    const int64_t rows = (int64_t)m.B * Hq * Tpad;
+    k_bwd_prep<<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(
+        (const __nv_bfloat16 *)o, (const __nv_bfloat16 *)dO, lse, m.B, m.N, Hq, Tpad, Drow, L2);
+    const float sl2 = scale * 1.4426950408889634f;
+    size_t smem = sizeof(DkvSmem) + 1024;
+    cudaError_t e = cudaFuncSetAttribute(k_attn_dkdv_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    k_attn_dkdv_tc<<<(unsigned)((int64_t)m.B * Hkv * m.T), kBwdThreads, smem, s>>>(
+        tq, tk, tv, to, m, Hq, Hkv, scale, sl2, Drow, L2, (__nv_bfloat16 *)dk, (__nv_bfloat16 *)dv,
+        status);
+    smem = sizeof(DqSmem) + 1024;
+    e = cudaFuncSetAttribute(k_attn_dq_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    k_attn_dq_tc<<<(unsigned)((int64_t)m.B * Hq * m.T), kBwdThreads, smem, s>>>(
+        tq, tk, tv, to, m, Hq, Hkv, scale, sl2, Drow, L2, (__nv_bfloat16 *)dq, status);
+    return cudaGetLastError();
+}
+
+}  // namespace kvs

@@ -378,3 +378,22 @@ def replay_tensors(cfg: TraceConfig, salt: int = 0):
     if cfg.dtype == "bf16":
         q, k, v, do = (round_bf16(t) for t in (q, k, v, do))
     return q, k, v, do
+
+
+def replay_tensors_device(cfg: TraceConfig, device="cuda", salt: int = 0, with_grad: bool = True):
+    """Full-size twin of :func:`replay_tensors` drawn with torch's CUDA generator
+    (same shapes and distribution, different stream); rounded to bf16 for bf16
+    configs. Returns (q, k, v, dO) as torch tensors on ``device``."""
+    import torch
+
+    g = torch.Generator(device=device)
+    g.manual_seed(cfg.seed(0) * 16 + salt)
+    B, N = cfg.batch, cfg.n_tokens
+    dt = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
+
+    def draw(h):
+        return torch.randn((B, N, h, cfg.d), generator=g, device=device, dtype=torch.float32).to(dt)
+
+    q, k, v = draw(cfg.hq), draw(cfg.hkv), draw(cfg.hkv)
+    do = draw(cfg.hq) if with_grad else None
+    return q, k, v, do

@@ -1,0 +1,156 @@
+"""GPU parity: eviction-masked attention forward and backward (fp32 CUDA-core
+path and bf16 tcgen05 path) against the fp64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import eviction_masked_attention_b200 as kvs
+from eviction_masked_attention_b200 import workloads as W
+from gpu_util import BF16_TOL, F32_TOL, GRAD_REL_L2, assert_close, dev, events_dev, host, rel_l2
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(cfg, ev, q, k, v, do, bwd=True):
+    tdt = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
+    gm = kvs.kvs_build_tile_mask(events_dev(ev), cfg.batch, cfg.n_tokens)
+    qd, kd, vd = dev(q, tdt), dev(k, tdt), dev(v, tdt)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    o, lse = kvs.kvs_masked_attn_fwd(qd, kd, vd, gm, cfg.scale, status=status)
+    out = dict(o=o, lse=lse, mask=gm)
+    if bwd:
+        dq, dk, dv = kvs.kvs_masked_attn_bwd(qd, kd, vd, o, dev(do, tdt), lse, gm, cfg.scale, status=status)
+        out.update(dq=dq, dk=dk, dv=dv)
+    torch.cuda.synchronize()
+    assert status.item() == 0, kvs.status_str(status.item())
+    return out
+
+
+def _check_full(cfg, ev, q, k, v, do, tol, bwd=True):
+    r = _run(cfg, ev, q, k, v, do, bwd)
+    kap = oracle.kappa(ev, cfg.batch, cfg.n_tokens)
+    if bwd:
+        o, lse, dq, dk, dv = oracle.attn_bwd(q, k, v, do, kap, cfg.scale)
+    else:
+        o, lse = oracle.attn_fwd(q, k, v, kap, cfg.scale)
+    assert_close(host(r["o"]), o, tol, "O")
+    assert_close(host(r["lse"]), lse, max(tol, 1e-5), "LSE")
+    if bwd:
+        for name, want in (("dq", dq), ("dk", dk), ("dv", dv)):
+            got = host(r[name])
+            assert_close(got, want, tol, name)
+            assert rel_l2(got, want) <= GRAD_REL_L2, (name, rel_l2(got, want))
+    return r
+
+
+def test_fp32_tiny_config_fwd_bwd():
+    cfg = W.CONFIGS[1]
+    ev = W.make_event_log(cfg)
+    q, k, v, do = W.replay_tensors(cfg)
+    _check_full(cfg, ev, q, k, v, do, F32_TOL)
+
+
+@pytest.mark.parametrize("cid,div,hq,hkv,batch", [
+    (2, 8, 8, 2, 2),      # recent-turns policy, GQA 4
+    (3, 16, 8, 2, 2),     # summary policy
+    (5, 32, 16, 2, 1),    # 1-token blocks, unpadded turns, GQA 8
+])
+def test_bf16_scaled_configs_fwd_bwd(cid, div, hq, hkv, batch):
+    cfg = W.replace(W.scaled(W.CONFIGS[cid], div), hq=hq, hkv=hkv, batch=batch)
+    ev = W.make_event_log(cfg)
+    assert len(ev) > 0
+    q, k, v, do = W.replay_tensors(cfg)
+    _check_full(cfg, ev, q, k, v, do, BF16_TOL)
+
+
+@pytest.mark.parametrize("N,dtype,seed", [(300, "bf16", 0), (1000, "bf16", 1), (129, "bf16", 2),
+                                          (1, "bf16", 3), (300, "f32", 4), (1000, "f32", 5)])
+def test_ragged_lengths_random_events(N, dtype, seed):
+    d = 128 if dtype == "bf16" else 64
+    cfg = W.TraceConfig(cid=90 + seed, name="ragged", batch=2, n_tokens=N, hq=4, hkv=2, d=d,
+                        theta=1e4, block_size=1, dtype=dtype, prompt=0)
+    ev = W.random_event_log(np.random.default_rng(seed), 2, N, 10, unit=1, max_span=max(1, N // 3))
+    q, k, v, do = W.replay_tensors(cfg)
+    _check_full(cfg, ev, q, k, v, do, BF16_TOL if dtype == "bf16" else F32_TOL)
+
+
+def test_bf16_no_events_and_mha():
+    cfg = W.TraceConfig(cid=80, name="mha", batch=1, n_tokens=640, hq=3, hkv=3, d=128, theta=1e4,
+                        block_size=1, dtype="bf16", prompt=0)
+    q, k, v, do = W.replay_tensors(cfg)
+    _check_full(cfg, np.zeros((0, 4), np.int32), q, k, v, do, BF16_TOL)
+
+
+def test_bf16_rope_then_attention_end_to_end():
+    # raw q, k -> logical RoPE -> masked attention, both sides from the same raw inputs
+    cfg = W.replace(W.scaled(W.CONFIGS[5], 64), hq=8, hkv=1, batch=1)
+    ev = W.make_event_log(cfg)
+    q, k, v, _ = W.replay_tensors(cfg)
+    N = cfg.n_tokens
+    lp = np.arange(N, dtype=np.int32)
+    qd = kvs.kvs_rope_logical(dev(q[0], torch.bfloat16), dev(lp), cfg.theta)[None]
+    kd = kvs.kvs_rope_logical(dev(k[0], torch.bfloat16), dev(lp), cfg.theta)[None]
+    gm = kvs.kvs_build_tile_mask(events_dev(ev), 1, N)
+    o, lse = kvs.kvs_masked_attn_fwd(qd.contiguous(), kd.contiguous(), dev(v, torch.bfloat16), gm, cfg.scale)
+    kap = oracle.kappa(ev, 1, N)
+    qo = oracle.rope(q[0], lp, cfg.theta)[None]
+    ko = oracle.rope(k[0], lp, cfg.theta)[None]
+    want, _ = oracle.attn_fwd(qo, ko, v.astype(np.float64), kap, cfg.scale)
+    assert_close(host(o), want, BF16_TOL, "rope+attn")
+
+
+# ------------------------------------------------------------------ full sizes (sampled)
+
+def _sample_rows(N, ev_b, rng, n=24):
+    taus = sorted(set(int(x) for x in ev_b[:, 1])) if len(ev_b) else []
+    cand = [0, 1, 127, 128, N - 1] + [t + o for t in taus for o in (-1, 0, 1) if 0 <= t + o < N]
+    cand += rng.integers(0, N, n).tolist()
+    return sorted(set(cand))
+
+
+@pytest.mark.parametrize("cid", [2, 3, 5])
+def test_full_size_sampled(cid):
+    cfg = W.CONFIGS[cid]
+    B, N, Hq, Hkv = cfg.batch, cfg.n_tokens, cfg.hq, cfg.hkv
+    G = Hq // Hkv
+    ev = W.make_event_log(cfg)
+    q, k, v, do = W.replay_tensors_device(cfg)
+    gm = kvs.kvs_build_tile_mask(events_dev(ev), B, N)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    o, lse = kvs.kvs_masked_attn_fwd(q, k, v, gm, cfg.scale, status=status)
+    bwd = cid in (3, 5)
+    if bwd:
+        dq, dk, dv = kvs.kvs_masked_attn_bwd(q, k, v, o, do, lse, gm, cfg.scale, status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    kap = oracle.kappa(ev, B, N)
+    rng = np.random.default_rng(cid)
+    for b in (0, B - 1):
+        rows = _sample_rows(N, ev[ev[:, 0] == b], rng)
+        for h in (0, Hq - 1):
+            kvh = h // G
+            kk, vv = host(k[b, :, kvh]), host(v[b, :, kvh])
+            want_o, want_l = oracle.attn_rows(host(q[b, rows, h]), rows, kk, vv, kap[b], cfg.scale)
+            assert_close(host(o[b, rows, h]), want_o, BF16_TOL, f"O b{b} h{h}")
+            assert_close(host(lse[b, h, rows]), want_l, BF16_TOL, f"LSE b{b} h{h}")
+            if bwd:
+                qg = host(q[b, :, kvh * G:(kvh + 1) * G].transpose(0, 1))
+                dg = host(do[b, :, kvh * G:(kvh + 1) * G].transpose(0, 1))
+                gr = np.full(len(rows), h - kvh * G)
+                want = oracle.dq_rows(qg, kk, vv, dg, kap[b], cfg.scale, gr, rows)
+                assert_close(host(dq[b, rows, h]), want, BF16_TOL, f"dQ b{b} h{h}")
+                cols = list(range(N - 8, N))
+                wk, wv = oracle.dkdv_cols(qg, kk, vv, dg, kap[b], cfg.scale, cols)
+                assert_close(host(dk[b, cols, kvh]), wk, BF16_TOL, f"dK b{b}")
+                assert_close(host(dv[b, cols, kvh]), wv, BF16_TOL, f"dV b{b}")
+    if bwd:
+        # properties at full size: sum_j dK_j = 0 and sum_j dV_j = sum over the group of dO_t
+        # (rows of P sum to 1; rows of dS sum to dO.(O - bf16(O)), a rounding-size term)
+        for b in (0, B - 1):
+            sdk = dk[b].double().sum(0)                        # [Hkv, d]
+            sdv = dv[b].double().sum(0)
+            sdo = do[b].double().sum(0).view(Hkv, G, -1).sum(1)
+            ek, ev_ = sdk.abs().max().item(), (sdv - sdo).abs().max().item()
+            print(f"cfg{cid} b{b}: |sum dK| {ek:.3g}, |sum dV - sum dO| {ev_:.3g}, |sum dO| {sdo.abs().max().item():.3g}")
+            assert ek <= 5.0 and ev_ <= 1.0
