@@ -24,6 +24,7 @@ LIB_PATH = os.path.join(_PKG, "libkvs.so")
 KVS_OK, KVS_ERR_INVALID_ARG, KVS_ERR_UNALIGNED, KVS_ERR_EVENT_ORDER = 0, 1, 2, 3
 KVS_ERR_CAPACITY, KVS_ERR_UNSUPPORTED, KVS_ERR_TIMEOUT, KVS_ERR_CUDA = 4, 5, 6, 7
 KVS_F32, KVS_BF16 = 0, 1
+KVS_BWD_PREP, KVS_BWD_DKDV, KVS_BWD_DQ, KVS_BWD_ALL = 1, 2, 4, 7
 TILE_EMPTY, TILE_FULL, TILE_PARTIAL = 0, 1, 2
 INT32_MAX = 2**31 - 1
 
@@ -31,14 +32,15 @@ EXPORTED = (
     "kvs_build_tile_mask_ws_bytes", "kvs_build_tile_mask", "kvs_compact_block_table",
     "kvs_rope_logical", "kvs_paged_decode_ws_bytes", "kvs_paged_decode_attn",
     "kvs_masked_attn_fwd", "kvs_masked_attn_bwd_ws_bytes", "kvs_masked_attn_bwd",
-    "kvs_status_str", "kvs_version",
+    "kvs_status_str", "kvs_version", "kvs_last_cuda_error",
 )
 
 
 class KvsError(RuntimeError):
     def __init__(self, code: int, where: str):
         self.code = code
-        super().__init__(f"{where}: {status_str(code)} (status {code})")
+        extra = f" [{lib().kvs_last_cuda_error().decode()}]" if code == KVS_ERR_CUDA else ""
+        super().__init__(f"{where}: {status_str(code)} (status {code}){extra}")
 
 
 class _TileMaskC(C.Structure):
@@ -78,14 +80,15 @@ def lib() -> C.CDLL:
         L.kvs_paged_decode_attn.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, i32,
                                             vp, vp, sz, vp, vp]
         L.kvs_masked_attn_fwd.argtypes = [vp, vp, vp, C.POINTER(_TileMaskC), i32, i32, i32, i32, i32,
-                                          f32, i32, vp, vp, vp, vp]
+                                          f32, i32, vp, vp, vp, vp, vp]
         L.kvs_masked_attn_bwd_ws_bytes.argtypes = [i32, i32, i32, i32, i32, i32]
         L.kvs_masked_attn_bwd_ws_bytes.restype = sz
-        L.kvs_masked_attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, C.POINTER(_TileMaskC), i32, i32, i32,
-                                          i32, i32, f32, i32, vp, vp, vp, vp, sz, vp, vp]
+        L.kvs_masked_attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, C.POINTER(_TileMaskC), i32, i32,
+                                          i32, i32, i32, f32, i32, vp, vp, vp, vp, sz, i32, vp, vp]
         L.kvs_status_str.argtypes = [i32]
         L.kvs_status_str.restype = C.c_char_p
         L.kvs_version.restype = i32
+        L.kvs_last_cuda_error.restype = C.c_char_p
         for r in ("kvs_build_tile_mask", "kvs_compact_block_table", "kvs_rope_logical",
                   "kvs_paged_decode_attn", "kvs_masked_attn_fwd", "kvs_masked_attn_bwd"):
             getattr(L, r).restype = i32
@@ -263,8 +266,11 @@ def kvs_paged_decode_attn(q, k_cache, v_cache, block_table, num_tokens, block_si
 
 # ------------------------------------------------------------------------------ attention
 
-def kvs_masked_attn_fwd(q, k, v, mask: TileMask, scale: float, out=None, lse=None, status=None):
-    """q [B, N, Hq, d], k/v [B, N, Hkv, d] -> (o [B, N, Hq, d], lse fp32 [B, Hq, N])."""
+def kvs_masked_attn_fwd(q, k, v, mask: TileMask, scale: float, out=None, lse=None, status=None,
+                        out_lo=None, residual: bool = True):
+    """q [B, N, Hq, d], k/v [B, N, Hkv, d] -> (o [B, N, Hq, d], lse fp32 [B, Hq, N], o_lo).
+    For bf16 with ``residual`` the rounding residual o_lo of the output is also
+    returned (pass it to the backward); otherwise o_lo is None."""
     _dev(q, k, v)
     B, N, Hq, d = q.shape
     Hkv = k.shape[2]
@@ -272,19 +278,24 @@ def kvs_masked_attn_fwd(q, k, v, mask: TileMask, scale: float, out=None, lse=Non
         out = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device)
+    if q.dtype == torch.bfloat16 and residual and out_lo is None:
+        out_lo = torch.empty_like(q)
+    if q.dtype != torch.bfloat16:
+        out_lo = None
     if status is None:
         status = torch.zeros(1, dtype=torch.int32, device=q.device)
     m = mask.c_struct()
     _check(lib().kvs_masked_attn_fwd(_p(q), _p(k), _p(v), C.byref(m), B, N, Hq, Hkv, d, float(scale),
-                                     _dtype_code(q), _p(out), _p(lse), _p(status), _stream()),
+                                     _dtype_code(q), _p(out), _p(out_lo), _p(lse), _p(status), _stream()),
            "kvs_masked_attn_fwd")
-    return out, lse
+    return out, lse, out_lo
 
 
 def kvs_masked_attn_bwd(q, k, v, o, do, lse, mask: TileMask, scale: float, dq=None, dk=None, dv=None,
-                        ws=None, status=None):
-    """Gradients (dq, dk, dv) of kvs_masked_attn_fwd."""
-    _dev(q, k, v, o, do, lse)
+                        ws=None, status=None, stages: int = KVS_BWD_ALL, o_lo=None):
+    """Gradients (dq, dk, dv) of kvs_masked_attn_fwd (``stages`` selects the kernels;
+    ``o_lo`` is the forward's output residual, improving D = <dO, O>)."""
+    _dev(q, k, v, o, do, lse, o_lo)
     B, N, Hq, d = q.shape
     Hkv = k.shape[2]
     L = lib()
@@ -298,7 +309,7 @@ def kvs_masked_attn_bwd(q, k, v, o, do, lse, mask: TileMask, scale: float, dq=No
     if status is None:
         status = torch.zeros(1, dtype=torch.int32, device=q.device)
     m = mask.c_struct()
-    _check(L.kvs_masked_attn_bwd(_p(q), _p(k), _p(v), _p(o), _p(do), _p(lse), C.byref(m), B, N, Hq, Hkv,
-                                 d, float(scale), dt, _p(dq), _p(dk), _p(dv), _p(ws), ws.numel(),
-                                 _p(status), _stream()), "kvs_masked_attn_bwd")
+    _check(L.kvs_masked_attn_bwd(_p(q), _p(k), _p(v), _p(o), _p(o_lo), _p(do), _p(lse), C.byref(m), B, N,
+                                 Hq, Hkv, d, float(scale), dt, _p(dq), _p(dk), _p(dv), _p(ws), ws.numel(),
+                                 int(stages), _p(status), _stream()), "kvs_masked_attn_bwd")
     return dq, dk, dv

@@ -5,12 +5,12 @@
 
 namespace kvs {
 cudaError_t launch_fwd_tc(const void *q, const void *k, const void *v, const kvs_tile_mask &m,
-                          int32_t Hq, int32_t Hkv, float scale, void *o, float *lse,
+                          int32_t Hq, int32_t Hkv, float scale, void *o, void *o_lo, float *lse,
                           int32_t *status, cudaStream_t s, bool *map_ok);
 cudaError_t launch_bwd_tc(const void *q, const void *k, const void *v, const void *o,
-                          const void *dO, const float *lse, const kvs_tile_mask &m, int32_t Hq,
+                          const void *o_lo, const void *dO, const float *lse, const kvs_tile_mask &m, int32_t Hq,
                           int32_t Hkv, float scale, void *dq, void *dk, void *dv, void *ws,
-                          int32_t *status, cudaStream_t s, bool *map_ok);
+                          int32_t stages, int32_t *status, cudaStream_t s, bool *map_ok);
 size_t bwd_tc_ws_bytes(int32_t B, int32_t N, int32_t Hq);
 cudaError_t launch_fwd_simt(const float *q, const float *k, const float *v, const kvs_tile_mask &m,
                             int32_t Hq, int32_t Hkv, int32_t d, float scale, float *o, float *lse,
@@ -48,23 +48,24 @@ static bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 extern "C" kvs_status kvs_masked_attn_fwd(const void *q, const void *k, const void *v,
                                           const kvs_tile_mask *m, int32_t B, int32_t N, int32_t Hq,
                                           int32_t Hkv, int32_t d, float scale, kvs_dtype dt,
-                                          void *o, float *lse, int32_t *dev_status,
+                                          void *o, void *o_lo, float *lse, int32_t *dev_status,
                                           kvs_stream_t stream) {
     kvs_status st = check_attn_args(m, B, N, Hq, Hkv, d, dt);
     if (st != KVS_OK) return st;
     if (!q || !k || !v || !o || !lse) return KVS_ERR_INVALID_ARG;
-    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return KVS_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(o_lo))
+        return KVS_ERR_INVALID_ARG;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     cudaError_t e;
     if (dt == KVS_BF16) {
         bool map_ok = false;
-        e = launch_fwd_tc(q, k, v, *m, Hq, Hkv, scale, o, lse, dev_status, s, &map_ok);
+        e = launch_fwd_tc(q, k, v, *m, Hq, Hkv, scale, o, o_lo, lse, dev_status, s, &map_ok);
         if (!map_ok) return KVS_ERR_INVALID_ARG;
     } else {
         e = launch_fwd_simt((const float *)q, (const float *)k, (const float *)v, *m, Hq, Hkv, d,
                             scale, (float *)o, lse, s);
     }
-    return e == cudaSuccess ? KVS_OK : KVS_ERR_CUDA;
+    return cuda_status(e);
 }
 
 extern "C" size_t kvs_masked_attn_bwd_ws_bytes(int32_t B, int32_t N, int32_t Hq, int32_t Hkv,
@@ -77,31 +78,34 @@ extern "C" size_t kvs_masked_attn_bwd_ws_bytes(int32_t B, int32_t N, int32_t Hq,
 }
 
 extern "C" kvs_status kvs_masked_attn_bwd(const void *q, const void *k, const void *v,
-                                          const void *o, const void *dO, const float *lse,
+                                          const void *o, const void *o_lo, const void *dO,
+                                          const float *lse,
                                           const kvs_tile_mask *m, int32_t B, int32_t N, int32_t Hq,
                                           int32_t Hkv, int32_t d, float scale, kvs_dtype dt,
                                           void *dq, void *dk, void *dv, void *ws, size_t ws_bytes,
-                                          int32_t *dev_status, kvs_stream_t stream) {
+                                          int32_t stages, int32_t *dev_status,
+                                          kvs_stream_t stream) {
     kvs_status st = check_attn_args(m, B, N, Hq, Hkv, d, dt);
     if (st != KVS_OK) return st;
     if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv || !ws) return KVS_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dO) ||
-        !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned16(ws))
+        !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned16(ws) || !aligned16(o_lo))
         return KVS_ERR_INVALID_ARG;
     if (ws_bytes < kvs_masked_attn_bwd_ws_bytes(B, N, Hq, Hkv, d, dt)) return KVS_ERR_CAPACITY;
+    if (stages <= 0 || stages > KVS_BWD_ALL) return KVS_ERR_INVALID_ARG;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     cudaError_t e;
     if (dt == KVS_BF16) {
         bool map_ok = false;
-        e = launch_bwd_tc(q, k, v, o, dO, lse, *m, Hq, Hkv, scale, dq, dk, dv, ws, dev_status, s,
-                          &map_ok);
+        e = launch_bwd_tc(q, k, v, o, o_lo, dO, lse, *m, Hq, Hkv, scale, dq, dk, dv, ws, stages,
+                          dev_status, s, &map_ok);
         if (!map_ok) return KVS_ERR_INVALID_ARG;
     } else {
         e = launch_bwd_simt((const float *)q, (const float *)k, (const float *)v, (const float *)o,
                             (const float *)dO, lse, *m, Hq, Hkv, d, scale, (float *)dq, (float *)dk,
                             (float *)dv, (float *)ws, s);
     }
-    return e == cudaSuccess ? KVS_OK : KVS_ERR_CUDA;
+    return cuda_status(e);
 }
 
 extern "C" const char *kvs_status_str(kvs_status s) {
@@ -119,3 +123,9 @@ extern "C" const char *kvs_status_str(kvs_status s) {
 }
 
 extern "C" int32_t kvs_version(void) { return 100; }
+
+thread_local const char *kvs::g_last_cuda_error = nullptr;
+
+extern "C" const char *kvs_last_cuda_error(void) {
+    return kvs::g_last_cuda_error ? kvs::g_last_cuda_error : "no error";
+}

@@ -26,7 +26,6 @@ namespace kvs {
 
 bool make_tmap_bnhd(CUtensorMap *map, const void *base, int B, int N, int H);
 
-constexpr int kBwdThreads = 192;
 constexpr uint32_t kTile = 128 * 128 * 2;
 
 __device__ __forceinline__ bool wait_done(uint64_t *bar, uint32_t parity) {
@@ -42,9 +41,11 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volati
 }
 
 // D[b][h][t] = <dO, O>, L2[b][h][t] = lse * log2(e); rows t >= N get 0. Tpad = T*128.
-__global__ void k_bwd_prep(const __nv_bfloat16 *__restrict__ o, const __nv_bfloat16 *__restrict__ dO,
-                           const float *__restrict__ lse, int32_t B, int32_t N, int32_t Hq,
-                           int32_t Tpad, float *__restrict__ Drow, float *__restrict__ L2) {
+// O is o_hi (+ o_lo when the forward kept the rounding residual of its output).
+__global__ void k_bwd_prep(const __nv_bfloat16 *__restrict__ o, const __nv_bfloat16 *__restrict__ o_lo,
+                           const __nv_bfloat16 *__restrict__ dO, const float *__restrict__ lse,
+                           int32_t B, int32_t N, int32_t Hq, int32_t Tpad, float *__restrict__ Drow,
+                           float *__restrict__ L2) {
     const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (row >= (int64_t)B * Hq * Tpad) return;
@@ -54,8 +55,12 @@ __global__ void k_bwd_prep(const __nv_bfloat16 *__restrict__ o, const __nv_bfloa
         const int64_t off = ((b * N + t) * Hq + h) * 128 + lane * 4;
         const uint2 a = *reinterpret_cast<const uint2 *>(o + off);
         const uint2 c = *reinterpret_cast<const uint2 *>(dO + off);
-        s = bf16_lo(a.x) * bf16_lo(c.x) + bf16_hi(a.x) * bf16_hi(c.x) + bf16_lo(a.y) * bf16_lo(c.y) +
-            bf16_hi(a.y) * bf16_hi(c.y);
+        float o0 = bf16_lo(a.x), o1 = bf16_hi(a.x), o2 = bf16_lo(a.y), o3 = bf16_hi(a.y);
+        if (o_lo) {
+            const uint2 r = *reinterpret_cast<const uint2 *>(o_lo + off);
+            o0 += bf16_lo(r.x); o1 += bf16_hi(r.x); o2 += bf16_lo(r.y); o3 += bf16_hi(r.y);
+        }
+        s = o0 * bf16_lo(c.x) + o1 * bf16_hi(c.x) + o2 * bf16_lo(c.y) + o3 * bf16_hi(c.y);
         for (int k = 16; k; k >>= 1) s += __shfl_xor_sync(0xffffffffu, s, k);
         l2 = lse[(b * Hq + h) * N + t] * 1.4426950408889634f;
     }
@@ -65,7 +70,31 @@ __global__ void k_bwd_prep(const __nv_bfloat16 *__restrict__ o, const __nv_bfloa
     }
 }
 
+// Store 64 fp32 values (times f) of a row as bf16 to 128 contiguous bytes.
+__device__ __forceinline__ void store_row64(__nv_bfloat16 *dst, const uint32_t (&a)[32],
+                                            const uint32_t (&b)[32], float f) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const uint32_t(&r)[32] = h ? b : a;
+#pragma unroll
+        for (int j = 0; j < 32; j += 8) {
+            uint4 w;
+            w.x = pack_bf16(__uint_as_float(r[j]) * f, __uint_as_float(r[j + 1]) * f);
+            w.y = pack_bf16(__uint_as_float(r[j + 2]) * f, __uint_as_float(r[j + 3]) * f);
+            w.z = pack_bf16(__uint_as_float(r[j + 4]) * f, __uint_as_float(r[j + 5]) * f);
+            w.w = pack_bf16(__uint_as_float(r[j + 6]) * f, __uint_as_float(r[j + 7]) * f);
+            *reinterpret_cast<uint4 *>(dst + h * 32 + j) = w;
+        }
+    }
+}
+
+// TMEM column of the packed bf16 A operand for K-step kk when each half of the
+// 128 K values was packed at the start of its own 64-column region.
+__device__ __forceinline__ uint32_t packed_col(int kk) { return (kk < 4) ? kk * 8 : 64 + (kk - 4) * 8; }
+
 // ---------------------------------------------------------------------- dK / dV
+
+constexpr int kBwdThreads = 320;  // warp 0 TMA, warp 1 MMA, warps 2..9 elementwise
 
 struct DkvSmem {
     uint8_t k[kTile];
@@ -108,8 +137,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         mbar_init(&S.st_full, 1);
         mbar_init(&S.dp_full, 1);
-        mbar_init(&S.p_ready, 128);
-        mbar_init(&S.ds_ready, 128);
+        mbar_init(&S.p_ready, 256);
+        mbar_init(&S.ds_ready, 256);
         mbar_init(&S.acc_done, 1);
         mbar_init(&S.fin, 1);
         S.abort = 0;
@@ -177,14 +206,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    mma_ts(tmem + cDV, tmem + cST + kk * 8, sw128_desc(oa + kk * 2048, kTile / 2, 1024),
-                           idMN, (n > 0 || kk > 0) ? 1u : 0u);
+                    mma_ts(tmem + cDV, tmem + cST + packed_col(kk),
+                           sw128_desc(oa + kk * 2048, kTile / 2, 1024), idMN, (n > 0 || kk > 0) ? 1u : 0u);
                 if (!mbar_wait(&S.ds_ready, n & 1, abort, status)) break;
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    mma_ts(tmem + cDK, tmem + cDP + kk * 8, sw128_desc(qa + kk * 2048, kTile / 2, 1024),
-                           idMN, (n > 0 || kk > 0) ? 1u : 0u);
+                    mma_ts(tmem + cDK, tmem + cDP + packed_col(kk),
+                           sw128_desc(qa + kk * 2048, kTile / 2, 1024), idMN, (n > 0 || kk > 0) ? 1u : 0u);
                 mma_commit(&S.empty[s]);
             }
             mma_commit(&S.acc_done);
@@ -192,10 +221,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             wait_done(&S.fin, 0);
         }
     } else {
-        const int quad = warp & 3;
-        const int c = quad * 32 + lane;  // key row within the tile
+        // thread = key row c (TMEM lane), half = which 64 query columns it handles
+        const int quad = warp & 3, half = (warp - 2) >> 2;
+        const int c = quad * 32 + lane;
         const int j = k0 + c;
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+        const uint32_t col0 = half * 64;
         const int32_t kap = j < N ? m.kappa[(int64_t)b * N + j] : 0;
         bool ok = true;
         for (int n = 0; n < nw; ++n) {
@@ -203,6 +234,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             const int e = n / G;
             const int q0 = m.col_row[c0 + e] * 128;
             const bool full = m.col_pidx[c0 + e] < 0;
+            // visible query rows of this key inside the tile: [rlo, rhi) (j <= t < kappa_j)
             int rlo = 0, rhi = 128;
             if (!full) {
                 if (j >= N) {
@@ -213,33 +245,39 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     rhi = (int)(hi < 0 ? 0 : (hi > 128 ? 128 : hi));
                 }
             }
+            rlo -= col0;
+            rhi -= col0;
             if (!warp_wait(&S.full[s], (n >> 1) & 1, abort, status) ||
                 !warp_wait(&S.st_full, n & 1, abort, status)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            float p[128];
+            float p[64];
             {
-                uint32_t r[4][32];
-#pragma unroll
-                for (int cc = 0; cc < 4; ++cc) tmem_ld32(tmem + lane_off + cST + cc * 32, r[cc]);
+                uint32_t r0[32], r1[32];
+                tmem_ld32(tmem + lane_off + cST + col0, r0);
+                tmem_ld32(tmem + lane_off + cST + col0 + 32, r1);
                 tmem_ld_wait();
+                const float4 *l2v = reinterpret_cast<const float4 *>(&S.l2[s][col0]);
 #pragma unroll
-                for (int cc = 0; cc < 4; ++cc)
+                for (int i = 0; i < 16; ++i) {
+                    const float4 lv = l2v[i];
+                    const float ls[4] = {lv.x, lv.y, lv.z, lv.w};
 #pragma unroll
-                    for (int jj = 0; jj < 32; ++jj) {
-                        const int rr = cc * 32 + jj;
-                        const float x = __uint_as_float(r[cc][jj]) * scale_log2 - S.l2[s][rr];
+                    for (int u = 0; u < 4; ++u) {
+                        const int rr = 4 * i + u;
+                        const uint32_t raw = rr < 32 ? r0[rr] : r1[rr - 32];
+                        const float x = __uint_as_float(raw) * scale_log2 - ls[u];
                         p[rr] = (rr >= rlo && rr < rhi) ? ex2(x) : 0.f;
                     }
+                }
             }
             {
-                uint32_t pk[2][32];
+                uint32_t pk[32];
 #pragma unroll
-                for (int rr = 0; rr < 128; rr += 2) pk[rr >> 6][(rr & 63) >> 1] = pack_bf16(p[rr], p[rr + 1]);
-                tmem_st32(tmem + lane_off + cST, pk[0]);
-                tmem_st32(tmem + lane_off + cST + 32, pk[1]);
+                for (int rr = 0; rr < 64; rr += 2) pk[rr >> 1] = pack_bf16(p[rr], p[rr + 1]);
+                tmem_st32(tmem + lane_off + cST + col0, pk);
             }
             tmem_st_wait();
             tc_fence_before();
@@ -249,23 +287,25 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 break;
             }
             tc_fence_after();
+            {
+                uint32_t r0[32], r1[32], pk[32];
+                tmem_ld32(tmem + lane_off + cDP + col0, r0);
+                tmem_ld32(tmem + lane_off + cDP + col0 + 32, r1);
+                tmem_ld_wait();
+                const float4 *ddv = reinterpret_cast<const float4 *>(&S.dd[s][col0]);
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                uint32_t pk[32];
+                for (int i = 0; i < 16; ++i) {
+                    const float4 dv4 = ddv[i];
+                    const float ds4[4] = {dv4.x, dv4.y, dv4.z, dv4.w};
 #pragma unroll
-                for (int cc = 0; cc < 2; ++cc) {
-                    uint32_t r[32];
-                    tmem_ld32(tmem + lane_off + cDP + (half * 2 + cc) * 32, r);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int jj = 0; jj < 32; jj += 2) {
-                        const int rr = (half * 2 + cc) * 32 + jj;
-                        const float d0 = p[rr] * (__uint_as_float(r[jj]) - S.dd[s][rr]);
-                        const float d1 = p[rr + 1] * (__uint_as_float(r[jj + 1]) - S.dd[s][rr + 1]);
-                        pk[cc * 16 + (jj >> 1)] = pack_bf16(d0, d1);
+                    for (int u = 0; u < 4; u += 2) {
+                        const int rr = 4 * i + u;
+                        const float a0 = __uint_as_float(rr < 32 ? r0[rr] : r1[rr - 32]);
+                        const float a1 = __uint_as_float(rr + 1 < 32 ? r0[rr + 1] : r1[rr + 1 - 32]);
+                        pk[rr >> 1] = pack_bf16(p[rr] * (a0 - ds4[u]), p[rr + 1] * (a1 - ds4[u + 1]));
                     }
                 }
-                tmem_st32(tmem + lane_off + cDP + half * 32, pk);
+                tmem_st32(tmem + lane_off + cDP + col0, pk);
             }
             tmem_st_wait();
             tc_fence_before();
@@ -273,33 +313,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         if (ok && nw > 0 && warp_wait(&S.acc_done, 0, abort, status)) {
             tc_fence_after();
-            const int64_t ro = (((int64_t)b * N + j) * Hkv + kvh) * 128;
+            const int64_t ro = (((int64_t)b * N + j) * Hkv + kvh) * 128 + col0;
 #pragma unroll
             for (int which = 0; which < 2; ++which) {
-                __nv_bfloat16 *dst = (which ? dk : dv) + ro;
-                const float f = which ? scale : 1.f;
-#pragma unroll
-                for (int cc = 0; cc < 4; ++cc) {
-                    uint32_t r[32];
-                    tmem_ld32(tmem + lane_off + (which ? cDK : cDV) + cc * 32, r);
-                    tmem_ld_wait();
-                    if (j < N) {
-#pragma unroll
-                        for (int jj = 0; jj < 32; jj += 8) {
-                            uint4 w;
-                            w.x = pack_bf16(__uint_as_float(r[jj]) * f, __uint_as_float(r[jj + 1]) * f);
-                            w.y = pack_bf16(__uint_as_float(r[jj + 2]) * f, __uint_as_float(r[jj + 3]) * f);
-                            w.z = pack_bf16(__uint_as_float(r[jj + 4]) * f, __uint_as_float(r[jj + 5]) * f);
-                            w.w = pack_bf16(__uint_as_float(r[jj + 6]) * f, __uint_as_float(r[jj + 7]) * f);
-                            *reinterpret_cast<uint4 *>(dst + cc * 32 + jj) = w;
-                        }
-                    }
-                }
+                uint32_t r0[32], r1[32];
+                const uint32_t cb = (which ? cDK : cDV) + col0;
+                tmem_ld32(tmem + lane_off + cb, r0);
+                tmem_ld32(tmem + lane_off + cb + 32, r1);
+                tmem_ld_wait();
+                if (j < N) store_row64((which ? dk : dv) + ro, r0, r1, which ? scale : 1.f);
             }
         } else if (nw == 0 && j < N) {
             // a key no query sees (cannot happen for a valid mask: the diagonal is visible)
-            const int64_t ro = (((int64_t)b * N + j) * Hkv + kvh) * 128;
-            for (int i = 0; i < 128; i += 8) {
+            const int64_t ro = (((int64_t)b * N + j) * Hkv + kvh) * 128 + col0;
+            for (int i = 0; i < 64; i += 8) {
                 *reinterpret_cast<uint4 *>(dk + ro + i) = make_uint4(0, 0, 0, 0);
                 *reinterpret_cast<uint4 *>(dv + ro + i) = make_uint4(0, 0, 0, 0);
             }
@@ -312,13 +339,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 }
 
 // ---------------------------------------------------------------------- dQ
+//
+// TMEM: S [0,128), dP [128,256), dQ accumulator [256,384), dS double buffer
+// [384,448) [448,512) (bf16 pairs). Because dS has its own buffers, S and dP of
+// the next key tile are issued as soon as the elementwise warps have read the
+// current ones, so the tensor core computes them while dS is being formed.
 
 struct DqSmem {
     uint8_t q[kTile];
     uint8_t dout[kTile];
     uint8_t k[2][kTile];
     uint8_t v[2][kTile];
-    uint64_t qo_full, full[2], empty[2], s_full, dp_full, ds_ready, acc_done, fin;
+    uint64_t qo_full, full[2], empty[2], s_full, dp_full, s_free, dp_free, ds_ready, dq_done,
+        acc_done, fin;
     uint32_t tmem_base;
     int abort;
 };
@@ -350,7 +383,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         mbar_init(&S.s_full, 1);
         mbar_init(&S.dp_full, 1);
-        mbar_init(&S.ds_ready, 128);
+        mbar_init(&S.s_free, 256);
+        mbar_init(&S.dp_free, 256);
+        mbar_init(&S.ds_ready, 256);
+        mbar_init(&S.dq_done, 1);
         mbar_init(&S.acc_done, 1);
         mbar_init(&S.fin, 1);
         S.abort = 0;
@@ -365,7 +401,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     tc_fence_after();
     const uint32_t tmem = S.tmem_base;
     volatile int *abort = &S.abort;
-    constexpr uint32_t cS = 0, cDP = 128, cDQ = 256;
+    constexpr uint32_t cS = 0, cDP = 128, cDQ = 256, cDS = 384;
 
     if (warp == 0) {
         if (lane == 0 && nt > 0) {
@@ -390,12 +426,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             const uint32_t idKM = idesc_bf16(128, 128, false, false);
             const uint32_t idMN = idesc_bf16(128, 128, false, true);
             const uint32_t qa = smem_u32(S.q), oa = smem_u32(S.dout);
-            bool ok = mbar_wait(&S.qo_full, 0, abort, status);
-            for (int n = 0; ok && n < nt; ++n) {
+            auto issue_s_dp = [&](int n) -> bool {
                 const int s = n & 1;
-                if (!mbar_wait(&S.full[s], (n >> 1) & 1, abort, status)) break;
-                tc_fence_after();
+                if (!mbar_wait(&S.full[s], (n >> 1) & 1, abort, status)) return false;
                 const uint32_t ka = smem_u32(S.k[s]), va = smem_u32(S.v[s]);
+                if (n > 0 && !mbar_wait(&S.s_free, (n - 1) & 1, abort, status)) return false;
+                tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint32_t off = (kk >> 2) * (kTile / 2) + (kk & 3) * 32;
@@ -403,6 +439,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                            idKM, kk > 0);
                 }
                 mma_commit(&S.s_full);
+                if (n > 0 && !mbar_wait(&S.dp_free, (n - 1) & 1, abort, status)) return false;
+                tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint32_t off = (kk >> 2) * (kTile / 2) + (kk & 3) * 32;
@@ -410,97 +448,102 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                            idKM, kk > 0);
                 }
                 mma_commit(&S.dp_full);
+                return true;
+            };
+            bool ok = mbar_wait(&S.qo_full, 0, abort, status) && issue_s_dp(0);
+            for (int n = 0; ok && n < nt; ++n) {
+                const int s = n & 1;
+                if (n + 1 < nt && !issue_s_dp(n + 1)) break;
                 if (!mbar_wait(&S.ds_ready, n & 1, abort, status)) break;
                 tc_fence_after();
+                const uint32_t ka = smem_u32(S.k[s]);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    mma_ts(tmem + cDQ, tmem + cS + kk * 8, sw128_desc(ka + kk * 2048, kTile / 2, 1024),
-                           idMN, (n > 0 || kk > 0) ? 1u : 0u);
+                    mma_ts(tmem + cDQ, tmem + cDS + s * 64 + kk * 8,
+                           sw128_desc(ka + kk * 2048, kTile / 2, 1024), idMN, (n > 0 || kk > 0) ? 1u : 0u);
                 mma_commit(&S.empty[s]);
+                mma_commit(&S.dq_done);
             }
             mma_commit(&S.acc_done);
             mma_commit(&S.fin);
             wait_done(&S.fin, 0);
         }
     } else {
-        const int quad = warp & 3;
+        // thread = query row (TMEM lane); half = which 64 key columns it handles
+        const int quad = warp & 3, half = (warp - 2) >> 2;
         const int row = quad * 32 + lane;
         const int t = q0 + row;
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+        const uint32_t col0 = half * 64;
         const int64_t ro = ((int64_t)b * Hq + hq) * Tpad + t;
         const float l2 = L2[ro], dd = Drow[ro];
         bool ok = true;
         for (int n = 0; n < nt; ++n) {
+            const int s = n & 1;
             const int32_t pid = m.row_pidx[e0 + n];
-            uint4 bits = make_uint4(~0u, ~0u, ~0u, ~0u);
+            uint2 bits = make_uint2(~0u, ~0u);
             if (pid >= 0)
-                bits = *reinterpret_cast<const uint4 *>(m.bits + (int64_t)pid * 512 + row * 4);
-            const uint32_t wb[4] = {bits.x, bits.y, bits.z, bits.w};
+                bits = *reinterpret_cast<const uint2 *>(m.bits + (int64_t)pid * 512 + row * 4 + half * 2);
             if (!warp_wait(&S.s_full, n & 1, abort, status)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            float p[128];
+            float p[64];
             {
-                uint32_t r[4][32];
-#pragma unroll
-                for (int cc = 0; cc < 4; ++cc) tmem_ld32(tmem + lane_off + cS + cc * 32, r[cc]);
+                uint32_t r0[32], r1[32];
+                tmem_ld32(tmem + lane_off + cS + col0, r0);
+                tmem_ld32(tmem + lane_off + cS + col0 + 32, r1);
                 tmem_ld_wait();
+                tc_fence_before();
+                mbar_arrive(&S.s_free);
 #pragma unroll
-                for (int cc = 0; cc < 4; ++cc)
-#pragma unroll
-                    for (int jj = 0; jj < 32; ++jj)
-                        p[cc * 32 + jj] = ((wb[cc] >> jj) & 1u)
-                                              ? ex2(__uint_as_float(r[cc][jj]) * scale_log2 - l2)
-                                              : 0.f;
+                for (int jj = 0; jj < 32; ++jj) {
+                    p[jj] = ((bits.x >> jj) & 1u) ? ex2(__uint_as_float(r0[jj]) * scale_log2 - l2) : 0.f;
+                    p[jj + 32] = ((bits.y >> jj) & 1u) ? ex2(__uint_as_float(r1[jj]) * scale_log2 - l2) : 0.f;
+                }
             }
             if (!warp_wait(&S.dp_full, n & 1, abort, status)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
+            uint32_t pk[32];
+            {
+                uint32_t r0[32], r1[32];
+                tmem_ld32(tmem + lane_off + cDP + col0, r0);
+                tmem_ld32(tmem + lane_off + cDP + col0 + 32, r1);
+                tmem_ld_wait();
+                tc_fence_before();
+                mbar_arrive(&S.dp_free);
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                uint32_t pk[32];
-#pragma unroll
-                for (int cc = 0; cc < 2; ++cc) {
-                    uint32_t r[32];
-                    tmem_ld32(tmem + lane_off + cDP + (half * 2 + cc) * 32, r);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int jj = 0; jj < 32; jj += 2) {
-                        const int kc = (half * 2 + cc) * 32 + jj;
-                        pk[cc * 16 + (jj >> 1)] = pack_bf16(p[kc] * (__uint_as_float(r[jj]) - dd),
-                                                            p[kc + 1] * (__uint_as_float(r[jj + 1]) - dd));
-                    }
+                for (int jj = 0; jj < 32; jj += 2) {
+                    pk[jj >> 1] = pack_bf16(p[jj] * (__uint_as_float(r0[jj]) - dd),
+                                            p[jj + 1] * (__uint_as_float(r0[jj + 1]) - dd));
+                    pk[16 + (jj >> 1)] = pack_bf16(p[jj + 32] * (__uint_as_float(r1[jj]) - dd),
+                                                   p[jj + 33] * (__uint_as_float(r1[jj + 1]) - dd));
                 }
-                tmem_st32(tmem + lane_off + cS + half * 32, pk);
             }
+            // dQ of item n-1 must be complete: its MMA has then consumed ds_ready
+            // phase n-1 (so this arrival cannot run two phases ahead) and the
+            // dS buffer written two items ago is free.
+            if (n >= 1 && !warp_wait(&S.dq_done, (n - 1) & 1, abort, status)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            tmem_st32(tmem + lane_off + cDS + s * 64 + half * 32, pk);
             tmem_st_wait();
             tc_fence_before();
             mbar_arrive(&S.ds_ready);
         }
         if (ok && nt > 0 && warp_wait(&S.acc_done, 0, abort, status)) {
             tc_fence_after();
-            __nv_bfloat16 *dst = dq + (((int64_t)b * N + t) * Hq + hq) * 128;
-#pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
-                uint32_t r[32];
-                tmem_ld32(tmem + lane_off + cDQ + cc * 32, r);
-                tmem_ld_wait();
-                if (t < N) {
-#pragma unroll
-                    for (int jj = 0; jj < 32; jj += 8) {
-                        uint4 w;
-                        w.x = pack_bf16(__uint_as_float(r[jj]) * scale, __uint_as_float(r[jj + 1]) * scale);
-                        w.y = pack_bf16(__uint_as_float(r[jj + 2]) * scale, __uint_as_float(r[jj + 3]) * scale);
-                        w.z = pack_bf16(__uint_as_float(r[jj + 4]) * scale, __uint_as_float(r[jj + 5]) * scale);
-                        w.w = pack_bf16(__uint_as_float(r[jj + 6]) * scale, __uint_as_float(r[jj + 7]) * scale);
-                        *reinterpret_cast<uint4 *>(dst + cc * 32 + jj) = w;
-                    }
-                }
-            }
+            uint32_t r0[32], r1[32];
+            tmem_ld32(tmem + lane_off + cDQ + col0, r0);
+            tmem_ld32(tmem + lane_off + cDQ + col0 + 32, r1);
+            tmem_ld_wait();
+            if (t < N) store_row64(dq + (((int64_t)b * N + t) * Hq + hq) * 128 + col0, r0, r1, scale);
         }
     }
     tc_fence_before();
@@ -515,9 +558,9 @@ size_t bwd_tc_ws_bytes(int32_t B, int32_t N, int32_t Hq) {
 }
 
 cudaError_t launch_bwd_tc(const void *q, const void *k, const void *v, const void *o,
-                          const void *dO, const float *lse, const kvs_tile_mask &m, int32_t Hq,
+                          const void *o_lo, const void *dO, const float *lse, const kvs_tile_mask &m, int32_t Hq,
                           int32_t Hkv, float scale, void *dq, void *dk, void *dv, void *ws,
-                          int32_t *status, cudaStream_t s, bool *map_ok) {
+                          int32_t stages, int32_t *status, cudaStream_t s, bool *map_ok) {
     CUtensorMap tq, tk, tv, to;
     *map_ok = make_tmap_bnhd(&tq, q, m.B, m.N, Hq) && make_tmap_bnhd(&tk, k, m.B, m.N, Hkv) &&
               make_tmap_bnhd(&tv, v, m.B, m.N, Hkv) && make_tmap_bnhd(&to, dO, m.B, m.N, Hq);
@@ -526,21 +569,29 @@ cudaError_t launch_bwd_tc(const void *q, const void *k, const void *v, const voi
     float *Drow = (float *)ws;
     float *L2 = Drow + (size_t)m.B * Hq * Tpad;
     const int64_t rows = (int64_t)m.B * Hq * Tpad;
-    k_bwd_prep<<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(
-        (const __nv_bfloat16 *)o, (const __nv_bfloat16 *)dO, lse, m.B, m.N, Hq, Tpad, Drow, L2);
+    if (stages & KVS_BWD_PREP)
+        k_bwd_prep<<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(
+            (const __nv_bfloat16 *)o, (const __nv_bfloat16 *)o_lo, (const __nv_bfloat16 *)dO, lse,
+            m.B, m.N, Hq, Tpad, Drow, L2);
     const float sl2 = scale * 1.4426950408889634f;
-    size_t smem = sizeof(DkvSmem) + 1024;
-    cudaError_t e = cudaFuncSetAttribute(k_attn_dkdv_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
-    if (e != cudaSuccess) return e;
-    k_attn_dkdv_tc<<<(unsigned)((int64_t)m.B * Hkv * m.T), kBwdThreads, smem, s>>>(
-        tq, tk, tv, to, m, Hq, Hkv, scale, sl2, Drow, L2, (__nv_bfloat16 *)dk, (__nv_bfloat16 *)dv,
-        status);
-    smem = sizeof(DqSmem) + 1024;
-    e = cudaFuncSetAttribute(k_attn_dq_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    k_attn_dq_tc<<<(unsigned)((int64_t)m.B * Hq * m.T), kBwdThreads, smem, s>>>(
-        tq, tk, tv, to, m, Hq, Hkv, scale, sl2, Drow, L2, (__nv_bfloat16 *)dq, status);
+    cudaError_t e = cudaSuccess;
+    if (stages & KVS_BWD_DKDV) {
+        const size_t smem = sizeof(DkvSmem) + 1024;
+        e = cudaFuncSetAttribute(k_attn_dkdv_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)smem);
+        if (e != cudaSuccess) return e;
+        k_attn_dkdv_tc<<<(unsigned)((int64_t)m.B * Hkv * m.T), kBwdThreads, smem, s>>>(
+            tq, tk, tv, to, m, Hq, Hkv, scale, sl2, Drow, L2, (__nv_bfloat16 *)dk,
+            (__nv_bfloat16 *)dv, status);
+    }
+    if (stages & KVS_BWD_DQ) {
+        const size_t smem = sizeof(DqSmem) + 1024;
+        e = cudaFuncSetAttribute(k_attn_dq_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)smem);
+        if (e != cudaSuccess) return e;
+        k_attn_dq_tc<<<(unsigned)((int64_t)m.B * Hq * m.T), kBwdThreads, smem, s>>>(
+            tq, tk, tv, to, m, Hq, Hkv, scale, sl2, Drow, L2, (__nv_bfloat16 *)dq, status);
+    }
     return cudaGetLastError();
 }
 

@@ -45,7 +45,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     k_attn_fwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, kvs_tile_mask m, int32_t Hq,
                   int32_t Hkv, float scale_log2, __nv_bfloat16 *__restrict__ out,
-                  float *__restrict__ lse, int32_t *status) {
+                  __nv_bfloat16 *__restrict__ out_lo, float *__restrict__ lse, int32_t *status) {
     extern __shared__ uint8_t smem_raw[];
     FwdSmem &S = *reinterpret_cast<FwdSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -232,7 +232,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             __all_sync(0xffffffffu, mbar_wait(&S.odone, (nt - 1) & 1, abort, status))) {
             tc_fence_after();
             const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-            __nv_bfloat16 *orow = out + (((int64_t)b * N + t) * Hq + hq) * 128;
+            const int64_t orow = (((int64_t)b * N + t) * Hq + hq) * 128;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 uint32_t o[32];
@@ -241,12 +241,293 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 if (t < N) {
 #pragma unroll
                     for (int j = 0; j < 32; j += 8) {
-                        uint4 w;
-                        w.x = pack_bf16(__uint_as_float(o[j]) * inv, __uint_as_float(o[j + 1]) * inv);
-                        w.y = pack_bf16(__uint_as_float(o[j + 2]) * inv, __uint_as_float(o[j + 3]) * inv);
-                        w.z = pack_bf16(__uint_as_float(o[j + 4]) * inv, __uint_as_float(o[j + 5]) * inv);
-                        w.w = pack_bf16(__uint_as_float(o[j + 6]) * inv, __uint_as_float(o[j + 7]) * inv);
-                        *reinterpret_cast<uint4 *>(orow + c * 32 + j) = w;
+                        uint32_t hi[4], lo[4];
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const float x0 = __uint_as_float(o[j + 2 * u]) * inv;
+                            const float x1 = __uint_as_float(o[j + 2 * u + 1]) * inv;
+                            hi[u] = pack_bf16(x0, x1);
+                            lo[u] = pack_bf16(x0 - bf16_lo(hi[u]), x1 - bf16_hi(hi[u]));
+                        }
+                        *reinterpret_cast<uint4 *>(out + orow + c * 32 + j) =
+                            make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                        if (out_lo)
+                            *reinterpret_cast<uint4 *>(out_lo + orow + c * 32 + j) =
+                                make_uint4(lo[0], lo[1], lo[2], lo[3]);
+                    }
+                }
+            }
+            if (t < N)
+                lse[((int64_t)b * Hq + hq) * N + t] =
+                    l_run > 0.f ? (m_run + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+// ------------------------------------------------------------------ two heads per CTA
+//
+// Used when the group size G is even: the CTA takes query heads h0 and h0+1 of
+// one kv group for the same query tile. Both heads share the tile list (the
+// mask does not depend on the head) and every K/V tile, so each K/V tile is
+// brought into shared memory once for two Q tiles. Two softmax warpgroups
+// (warps 2..5 for h0, 6..9 for h0+1) alternate with the tensor core, which is
+// fed in the order S0_n, S1_n, PV0_n, S0_{n+1}, PV1_n, S1_{n+1}, ...
+// TMEM: S0 [0,128), S1 [128,256), O0 [256,384), O1 [384,512).
+
+constexpr int kFwd2Threads = 320;
+
+struct Fwd2Smem {
+    uint8_t q[2][kTileBytes];
+    uint8_t k[2][kTileBytes];
+    uint8_t v[2][kTileBytes];
+    uint64_t bar_q, kfull[2], kempty[2], vfull[2], vempty[2], sfull[2], pfull[2], odone[2], fin;
+    uint32_t tmem_base;
+    int abort;
+};
+
+__global__ void __launch_bounds__(kFwd2Threads, 1)
+    k_attn_fwd_tc2(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV, kvs_tile_mask m, int32_t Hq,
+                   int32_t Hkv, float scale_log2, __nv_bfloat16 *__restrict__ out,
+                   __nv_bfloat16 *__restrict__ out_lo, float *__restrict__ lse, int32_t *status) {
+    extern __shared__ uint8_t smem_raw[];
+    Fwd2Smem &S = *reinterpret_cast<Fwd2Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~uintptr_t(1023));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int B = m.B, N = m.N, T = m.T, G = Hq / Hkv, HP = Hq / 2;
+    const int64_t idx = blockIdx.x;
+    const int qi = T - 1 - (int)(idx / ((int64_t)B * HP));
+    const int rem = (int)(idx % ((int64_t)B * HP));
+    const int h0 = 2 * (rem % HP), b = rem / HP, kvh = h0 / G;
+    const int q0 = qi * 128;
+    const int32_t e0 = m.row_ptr[b * T + qi], nt = m.row_ptr[b * T + qi + 1] - e0;
+    if (grid_timed_out(status)) return;
+
+    if (threadIdx.x == 0) {
+        mbar_init(&S.bar_q, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&S.kfull[i], 1);
+            mbar_init(&S.kempty[i], 1);
+            mbar_init(&S.vfull[i], 1);
+            mbar_init(&S.vempty[i], 1);
+            mbar_init(&S.sfull[i], 1);
+            mbar_init(&S.pfull[i], 128);
+            mbar_init(&S.odone[i], 1);
+        }
+        mbar_init(&S.fin, 1);
+        S.abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(&S.tmem_base, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = S.tmem_base;
+    volatile int *abort = &S.abort;
+
+    if (warp == 0) {
+        if (lane == 0 && nt > 0) {
+            tma_prefetch_desc(&tmQ);
+            tma_prefetch_desc(&tmK);
+            tma_prefetch_desc(&tmV);
+            mbar_expect_tx(&S.bar_q, 2 * kTileBytes);
+            for (int x = 0; x < 2; ++x) {
+                tma_load_4d(S.q[x], &tmQ, &S.bar_q, 0, h0 + x, q0, b);
+                tma_load_4d(S.q[x] + kTileBytes / 2, &tmQ, &S.bar_q, 64, h0 + x, q0, b);
+            }
+            for (int n = 0; n < nt; ++n) {
+                const int s = n & 1;
+                const uint32_t ph = ((n >> 1) - 1) & 1;
+                const int k0 = m.row_col[e0 + n] * 128;
+                if (n >= 2 && !mbar_wait(&S.kempty[s], ph, abort, status)) break;
+                mbar_expect_tx(&S.kfull[s], kTileBytes);
+                tma_load_4d(S.k[s], &tmK, &S.kfull[s], 0, kvh, k0, b);
+                tma_load_4d(S.k[s] + kTileBytes / 2, &tmK, &S.kfull[s], 64, kvh, k0, b);
+                if (n >= 2 && !mbar_wait(&S.vempty[s], ph, abort, status)) break;
+                mbar_expect_tx(&S.vfull[s], kTileBytes);
+                tma_load_4d(S.v[s], &tmV, &S.vfull[s], 0, kvh, k0, b);
+                tma_load_4d(S.v[s] + kTileBytes / 2, &tmV, &S.vfull[s], 64, kvh, k0, b);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && nt > 0) {
+            const uint32_t idS = idesc_bf16(128, 128, false, false);
+            const uint32_t idPV = idesc_bf16(128, 128, false, true);
+            auto issue_s = [&](int x, int n) {
+                const uint32_t qa = smem_u32(S.q[x]), ka = smem_u32(S.k[n & 1]);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t off = (kk >> 2) * (kTileBytes / 2) + (kk & 3) * 32;
+                    mma_ss(tmem + x * 128, sw128_desc(qa + off, 16, 1024),
+                           sw128_desc(ka + off, 16, 1024), idS, kk > 0);
+                }
+                mma_commit(&S.sfull[x]);
+            };
+            auto issue_pv = [&](int x, int n) {
+                const uint32_t va = smem_u32(S.v[n & 1]);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_ts(tmem + 256 + x * 128, tmem + x * 128 + kk * 8,
+                           sw128_desc(va + kk * 2048, kTileBytes / 2, 1024), idPV,
+                           (n > 0 || kk > 0) ? 1u : 0u);
+                mma_commit(&S.odone[x]);
+            };
+            bool ok = mbar_wait(&S.bar_q, 0, abort, status) &&
+                      mbar_wait(&S.kfull[0], 0, abort, status);
+            if (ok) {
+                tc_fence_after();
+                issue_s(0, 0);
+                issue_s(1, 0);
+                mma_commit(&S.kempty[0]);
+            }
+            for (int n = 0; ok && n < nt; ++n) {
+                const int s = n & 1;
+                const bool more = n + 1 < nt;
+                if (!mbar_wait(&S.pfull[0], n & 1, abort, status)) break;
+                if (!mbar_wait(&S.vfull[s], (n >> 1) & 1, abort, status)) break;
+                tc_fence_after();
+                issue_pv(0, n);
+                if (more) {
+                    if (!mbar_wait(&S.kfull[(n + 1) & 1], ((n + 1) >> 1) & 1, abort, status)) break;
+                    tc_fence_after();
+                    issue_s(0, n + 1);
+                }
+                if (!mbar_wait(&S.pfull[1], n & 1, abort, status)) break;
+                tc_fence_after();
+                issue_pv(1, n);
+                mma_commit(&S.vempty[s]);
+                if (more) {
+                    issue_s(1, n + 1);
+                    mma_commit(&S.kempty[(n + 1) & 1]);
+                }
+            }
+            mma_commit(&S.fin);
+            wait_final(&S.fin, 0);
+        }
+    } else {
+        const int x = (warp - 2) >> 2;           // which head of the pair
+        const int quad = warp & 3;
+        const int row = quad * 32 + lane;
+        const int t = q0 + row;
+        const int hq = h0 + x;
+        const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+        const uint32_t cS = x * 128, cO = 256 + x * 128;
+        float m_run = -INFINITY, l_run = 0.f;
+        bool ok = true;
+        for (int n = 0; n < nt; ++n) {
+            const int32_t pid = m.row_pidx[e0 + n];
+            uint4 bits = make_uint4(~0u, ~0u, ~0u, ~0u);
+            if (pid >= 0)
+                bits = *reinterpret_cast<const uint4 *>(m.bits + (int64_t)pid * 512 + row * 4);
+            if (!__all_sync(0xffffffffu, mbar_wait(&S.sfull[x], n & 1, abort, status))) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t wb[4] = {bits.x, bits.y, bits.z, bits.w};
+            // pass 1: row maximum of the masked, base-2 scaled scores
+            float mt = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                uint32_t r[32];
+                tmem_ld32(tmem + lane_off + cS + c * 32, r);
+                tmem_ld_wait();
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                    if ((wb[c] >> j) & 1u) mt = fmaxf(mt, __uint_as_float(r[j]) * scale_log2);
+            }
+            const float m_new = fmaxf(m_run, mt);
+            float alpha = 1.f;
+            bool rescale = false;
+            if (m_run == -INFINITY) {
+                m_run = m_new;
+            } else if (m_new > m_run + kRescaleThreshold) {
+                alpha = ex2(m_run - m_new);
+                m_run = m_new;
+                l_run *= alpha;
+                rescale = true;
+            }
+            if (__any_sync(0xffffffffu, rescale) && n > 0) {
+                if (!__all_sync(0xffffffffu, mbar_wait(&S.odone[x], (n - 1) & 1, abort, status))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+#pragma unroll 1
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t o[32];
+                    tmem_ld32(tmem + lane_off + cO + c * 32, o);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+                    tmem_st32(tmem + lane_off + cO + c * 32, o);
+                }
+            }
+            // pass 2: P = 2^(s - m) as bf16 pairs over the first 64 columns of S
+            // (two 32-column score chunks are read before their 32 packed columns
+            // are written over the first of them)
+            const float mref = m_run == -INFINITY ? 0.f : m_run;
+            float lsum = 0.f;
+#pragma unroll 1
+            for (int hc = 0; hc < 2; ++hc) {
+                uint32_t pk[32];
+#pragma unroll
+                for (int cc = 0; cc < 2; ++cc) {
+                    const int c = 2 * hc + cc;
+                    const uint32_t w = hc ? (cc ? wb[3] : wb[2]) : (cc ? wb[1] : wb[0]);
+                    uint32_t r[32];
+                    tmem_ld32(tmem + lane_off + cS + c * 32, r);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int j = 0; j < 32; j += 2) {
+                        const float s0 = __uint_as_float(r[j]) * scale_log2 - mref;
+                        const float s1 = __uint_as_float(r[j + 1]) * scale_log2 - mref;
+                        const float p0 = ((w >> j) & 1u) ? ex2(s0) : 0.f;
+                        const float p1 = ((w >> (j + 1)) & 1u) ? ex2(s1) : 0.f;
+                        lsum += p0 + p1;
+                        pk[cc * 16 + (j >> 1)] = pack_bf16(p0, p1);
+                    }
+                }
+                tmem_st32(tmem + lane_off + cS + hc * 32, pk);
+            }
+            l_run += lsum;
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(&S.pfull[x]);
+        }
+        if (ok && nt > 0 &&
+            __all_sync(0xffffffffu, mbar_wait(&S.odone[x], (nt - 1) & 1, abort, status))) {
+            tc_fence_after();
+            const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+            const int64_t orow = (((int64_t)b * N + t) * Hq + hq) * 128;
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+                uint32_t o[32];
+                tmem_ld32(tmem + lane_off + cO + c * 32, o);
+                tmem_ld_wait();
+                if (t < N) {
+#pragma unroll
+                    for (int j = 0; j < 32; j += 8) {
+                        uint32_t hi[4], lo[4];
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const float x0 = __uint_as_float(o[j + 2 * u]) * inv;
+                            const float x1 = __uint_as_float(o[j + 2 * u + 1]) * inv;
+                            hi[u] = pack_bf16(x0, x1);
+                            lo[u] = pack_bf16(x0 - bf16_lo(hi[u]), x1 - bf16_hi(hi[u]));
+                        }
+                        *reinterpret_cast<uint4 *>(out + orow + c * 32 + j) =
+                            make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                        if (out_lo)
+                            *reinterpret_cast<uint4 *>(out_lo + orow + c * 32 + j) =
+                                make_uint4(lo[0], lo[1], lo[2], lo[3]);
                     }
                 }
             }
@@ -296,20 +577,31 @@ bool make_tmap_bnhd(CUtensorMap *map, const void *base, int B, int N, int H) {
 }
 
 cudaError_t launch_fwd_tc(const void *q, const void *k, const void *v, const kvs_tile_mask &m,
-                          int32_t Hq, int32_t Hkv, float scale, void *o, float *lse,
+                          int32_t Hq, int32_t Hkv, float scale, void *o, void *o_lo, float *lse,
                           int32_t *status, cudaStream_t s, bool *map_ok) {
     CUtensorMap tq, tk, tv;
     *map_ok = make_tmap_bnhd(&tq, q, m.B, m.N, Hq) && make_tmap_bnhd(&tk, k, m.B, m.N, Hkv) &&
               make_tmap_bnhd(&tv, v, m.B, m.N, Hkv);
     if (!*map_ok) return cudaSuccess;
-    const size_t smem = sizeof(FwdSmem) + 1024;
-    cudaError_t e =
-        cudaFuncSetAttribute(k_attn_fwd_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    const int64_t grid = (int64_t)m.B * Hq * m.T;
-    k_attn_fwd_tc<<<(unsigned)grid, kFwdThreads, smem, s>>>(tq, tk, tv, m, Hq, Hkv,
-                                                            scale * 1.4426950408889634f,
-                                                            (__nv_bfloat16 *)o, lse, status);
+    const int G = Hq / Hkv;
+    const float sl2 = scale * 1.4426950408889634f;
+    if (G % 2 == 0) {
+        const size_t smem = sizeof(Fwd2Smem) + 1024;
+        cudaError_t e = cudaFuncSetAttribute(k_attn_fwd_tc2, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)smem);
+        if (e != cudaSuccess) return e;
+        const int64_t grid = (int64_t)m.B * (Hq / 2) * m.T;
+        k_attn_fwd_tc2<<<(unsigned)grid, kFwd2Threads, smem, s>>>(
+            tq, tk, tv, m, Hq, Hkv, sl2, (__nv_bfloat16 *)o, (__nv_bfloat16 *)o_lo, lse, status);
+    } else {
+        const size_t smem = sizeof(FwdSmem) + 1024;
+        cudaError_t e = cudaFuncSetAttribute(k_attn_fwd_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)smem);
+        if (e != cudaSuccess) return e;
+        const int64_t grid = (int64_t)m.B * Hq * m.T;
+        k_attn_fwd_tc<<<(unsigned)grid, kFwdThreads, smem, s>>>(
+            tq, tk, tv, m, Hq, Hkv, sl2, (__nv_bfloat16 *)o, (__nv_bfloat16 *)o_lo, lse, status);
+    }
     return cudaGetLastError();
 }
 

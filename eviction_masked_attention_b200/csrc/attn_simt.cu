@@ -8,8 +8,10 @@
 // trainer replay; "KV-streams for Efficient Compaction in Agentic
 // Reinforcement Learning", Fig. 2(A).)
 //
-// Thread layout: SPLIT = D/32 threads per row, each owning 32 consecutive
-// feature dims; dot products are reduced over the SPLIT lanes.
+// Thread layout: SPLIT = D/16 threads per row, each owning 16 consecutive
+// feature dims; dot products are reduced over the SPLIT lanes. Long sums (the
+// output rows, the softmax denominator, dQ, dK, dV) use compensated (Kahan)
+// accumulation so fp32 rounding does not grow with the number of visible keys.
 #include "common.cuh"
 
 namespace kvs {
@@ -20,6 +22,23 @@ __device__ __forceinline__ float group_sum(float x) {
     for (int o = 1; o < SPLIT; o <<= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
     return x;
 }
+
+// Kahan-compensated running sum.
+struct KSum {
+    float s = 0.f, c = 0.f;
+    __device__ __forceinline__ void add(float x) {
+        const float y = x - c;
+        const float t = s + y;
+        c = (t - s) - y;
+        s = t;
+    }
+    __device__ __forceinline__ void scale(float a) {
+        s *= a;
+        c *= a;
+    }
+};
+
+constexpr int kDims = 16;  // feature dims owned by one thread
 
 __device__ __forceinline__ bool tile_bit(const uint32_t *bits_row, int c) {
     return (bits_row[c >> 5] >> (c & 31)) & 1u;
@@ -39,11 +58,11 @@ __device__ void load_tile(float *dst, const float *src_b, int32_t N, int32_t H, 
 }
 
 template <int D>
-__global__ void __launch_bounds__(128 * (D / 32), 1)
+__global__ void __launch_bounds__(128 * (D / kDims), 1)
     k_fwd_simt(const float *__restrict__ q, const float *__restrict__ k,
                const float *__restrict__ v, kvs_tile_mask m, int32_t Hq, int32_t Hkv,
                float scale, float *__restrict__ o, float *__restrict__ lse) {
-    constexpr int SPLIT = D / 32;
+    constexpr int SPLIT = D / kDims;
     extern __shared__ __align__(16) float sm[];
     float *sK = sm, *sV = sm + 128 * D;
     __shared__ uint32_t sBits[128][4];
@@ -52,14 +71,12 @@ __global__ void __launch_bounds__(128 * (D / 32), 1)
     const int r = threadIdx.x / SPLIT, part = threadIdx.x % SPLIT;
     const int t = qi * 128 + r;
     const bool live = t < N;
-    float qr[32], acc[32];
-    const float *qrow = q + (((int64_t)b * N + (live ? t : 0)) * Hq + h) * D + part * 32;
+    float qr[kDims];
+    KSum acc[kDims], l;
+    const float *qrow = q + (((int64_t)b * N + (live ? t : 0)) * Hq + h) * D + part * kDims;
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-        qr[i] = live ? qrow[i] * scale : 0.f;
-        acc[i] = 0.f;
-    }
-    float mx = -INFINITY, l = 0.f;
+    for (int i = 0; i < kDims; ++i) qr[i] = live ? qrow[i] * scale : 0.f;
+    float mx = -INFINITY;
     const float *kb = k + (int64_t)b * N * Hkv * D, *vb = v + (int64_t)b * N * Hkv * D;
     const int32_t e0 = m.row_ptr[b * T + qi], e1 = m.row_ptr[b * T + qi + 1];
     for (int32_t e = e0; e < e1; ++e) {
@@ -73,33 +90,34 @@ __global__ void __launch_bounds__(128 * (D / 32), 1)
         __syncthreads();
         for (int c = 0; c < 128; ++c) {
             float s = 0.f;
-            const float *kr = sK + c * D + part * 32;
+            const float *kr = sK + c * D + part * kDims;
 #pragma unroll
-            for (int i = 0; i < 32; ++i) s = fmaf(qr[i], kr[i], s);
+            for (int i = 0; i < kDims; ++i) s = fmaf(qr[i], kr[i], s);
             s = group_sum<SPLIT>(s);
             const bool vis = live && (pid < 0 || tile_bit(sBits[r], c));
             if (!vis) continue;
-            const float *vr = sV + c * D + part * 32;
+            const float *vr = sV + c * D + part * kDims;
+            float p = 1.f;
             if (s > mx) {
                 const float alpha = expf(mx - s);
-                l = l * alpha + 1.f;
+                l.scale(alpha);
 #pragma unroll
-                for (int i = 0; i < 32; ++i) acc[i] = fmaf(acc[i], alpha, vr[i]);
+                for (int i = 0; i < kDims; ++i) acc[i].scale(alpha);
                 mx = s;
             } else {
-                const float p = expf(s - mx);
-                l += p;
-#pragma unroll
-                for (int i = 0; i < 32; ++i) acc[i] = fmaf(p, vr[i], acc[i]);
+                p = expf(s - mx);
             }
+            l.add(p);
+#pragma unroll
+            for (int i = 0; i < kDims; ++i) acc[i].add(p * vr[i]);
         }
     }
     if (!live) return;
-    const float inv = l > 0.f ? 1.f / l : 0.f;
-    float *orow = o + (((int64_t)b * N + t) * Hq + h) * D + part * 32;
+    const float lsum = l.s;
+    float *orow = o + (((int64_t)b * N + t) * Hq + h) * D + part * kDims;
 #pragma unroll
-    for (int i = 0; i < 32; ++i) orow[i] = acc[i] * inv;
-    if (part == 0) lse[((int64_t)b * Hq + h) * N + t] = l > 0.f ? mx + logf(l) : -INFINITY;
+    for (int i = 0; i < kDims; ++i) orow[i] = lsum > 0.f ? acc[i].s / lsum : 0.f;
+    if (part == 0) lse[((int64_t)b * Hq + h) * N + t] = lsum > 0.f ? mx + logf(lsum) : -INFINITY;
 }
 
 // D_t = <dO_t, O_t> (fp32), one warp per row.
@@ -120,12 +138,12 @@ __global__ void k_rowdot_f32(const float *__restrict__ o, const float *__restric
 }
 
 template <int D>
-__global__ void __launch_bounds__(128 * (D / 32), 1)
+__global__ void __launch_bounds__(128 * (D / kDims), 1)
     k_dq_simt(const float *__restrict__ q, const float *__restrict__ k,
               const float *__restrict__ v, const float *__restrict__ dO,
               const float *__restrict__ lse, const float *__restrict__ Drow, kvs_tile_mask m,
               int32_t Hq, int32_t Hkv, float scale, float *__restrict__ dq) {
-    constexpr int SPLIT = D / 32;
+    constexpr int SPLIT = D / kDims;
     extern __shared__ __align__(16) float sm[];
     float *sK = sm, *sV = sm + 128 * D;
     __shared__ uint32_t sBits[128][4];
@@ -134,13 +152,13 @@ __global__ void __launch_bounds__(128 * (D / 32), 1)
     const int r = threadIdx.x / SPLIT, part = threadIdx.x % SPLIT;
     const int t = qi * 128 + r;
     const bool live = t < N;
-    float qr[32], dor[32], acc[32];
-    const int64_t rowoff = (((int64_t)b * N + (live ? t : 0)) * Hq + h) * D + part * 32;
+    float qr[kDims], dor[kDims];
+    KSum acc[kDims];
+    const int64_t rowoff = (((int64_t)b * N + (live ? t : 0)) * Hq + h) * D + part * kDims;
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
+    for (int i = 0; i < kDims; ++i) {
         qr[i] = live ? q[rowoff + i] : 0.f;
         dor[i] = live ? dO[rowoff + i] : 0.f;
-        acc[i] = 0.f;
     }
     const float L = live ? lse[((int64_t)b * Hq + h) * N + t] : 0.f;
     const float Dt = live ? Drow[((int64_t)b * Hq + h) * N + t] : 0.f;
@@ -156,10 +174,10 @@ __global__ void __launch_bounds__(128 * (D / 32), 1)
                 sBits[i >> 2][i & 3] = m.bits[(int64_t)pid * 512 + i];
         __syncthreads();
         for (int c = 0; c < 128; ++c) {
-            const float *kr = sK + c * D + part * 32, *vr = sV + c * D + part * 32;
+            const float *kr = sK + c * D + part * kDims, *vr = sV + c * D + part * kDims;
             float s = 0.f, dp = 0.f;
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
+            for (int i = 0; i < kDims; ++i) {
                 s = fmaf(qr[i], kr[i], s);
                 dp = fmaf(dor[i], vr[i], dp);
             }
@@ -170,23 +188,23 @@ __global__ void __launch_bounds__(128 * (D / 32), 1)
             const float p = expf(s * scale - L);
             const float ds = p * (dp - Dt);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) acc[i] = fmaf(ds, kr[i], acc[i]);
+            for (int i = 0; i < kDims; ++i) acc[i].add(ds * kr[i]);
         }
     }
     if (!live) return;
     float *out = dq + rowoff;
 #pragma unroll
-    for (int i = 0; i < 32; ++i) out[i] = acc[i] * scale;
+    for (int i = 0; i < kDims; ++i) out[i] = acc[i].s * scale;
 }
 
 template <int D>
-__global__ void __launch_bounds__(128 * (D / 32), 1)
+__global__ void __launch_bounds__(128 * (D / kDims), 1)
     k_dkdv_simt(const float *__restrict__ q, const float *__restrict__ k,
                 const float *__restrict__ v, const float *__restrict__ dO,
                 const float *__restrict__ lse, const float *__restrict__ Drow, kvs_tile_mask m,
                 int32_t Hq, int32_t Hkv, float scale, float *__restrict__ dk,
                 float *__restrict__ dv) {
-    constexpr int SPLIT = D / 32;
+    constexpr int SPLIT = D / kDims;
     extern __shared__ __align__(16) float sm[];
     float *sQ = sm, *sO = sm + 128 * D;
     __shared__ uint32_t sBits[128][4];
@@ -196,13 +214,13 @@ __global__ void __launch_bounds__(128 * (D / 32), 1)
     const int c = threadIdx.x / SPLIT, part = threadIdx.x % SPLIT;
     const int j = kj * 128 + c;
     const bool live = j < N;
-    float kr[32], vr[32], adk[32], adv[32];
-    const int64_t rowoff = (((int64_t)b * N + (live ? j : 0)) * Hkv + kvh) * D + part * 32;
+    float kr[kDims], vr[kDims];
+    KSum adk[kDims], adv[kDims];
+    const int64_t rowoff = (((int64_t)b * N + (live ? j : 0)) * Hkv + kvh) * D + part * kDims;
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
+    for (int i = 0; i < kDims; ++i) {
         kr[i] = live ? k[rowoff + i] : 0.f;
         vr[i] = live ? v[rowoff + i] : 0.f;
-        adk[i] = adv[i] = 0.f;
     }
     const float *qb = q + (int64_t)b * N * Hq * D, *ob = dO + (int64_t)b * N * Hq * D;
     const int32_t e0 = m.col_ptr[b * T + kj], e1 = m.col_ptr[b * T + kj + 1];
@@ -223,10 +241,10 @@ __global__ void __launch_bounds__(128 * (D / 32), 1)
                     sBits[i >> 2][i & 3] = m.bits[(int64_t)pid * 512 + i];
             __syncthreads();
             for (int r = 0; r < 128; ++r) {
-                const float *qr = sQ + r * D + part * 32, *dr = sO + r * D + part * 32;
+                const float *qr = sQ + r * D + part * kDims, *dr = sO + r * D + part * kDims;
                 float s = 0.f, dp = 0.f;
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
+                for (int i = 0; i < kDims; ++i) {
                     s = fmaf(qr[i], kr[i], s);
                     dp = fmaf(dr[i], vr[i], dp);
                 }
@@ -237,18 +255,18 @@ __global__ void __launch_bounds__(128 * (D / 32), 1)
                 const float p = expf(s * scale - sL[r]);
                 const float ds = p * (dp - sD[r]);
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    adv[i] = fmaf(p, dr[i], adv[i]);
-                    adk[i] = fmaf(ds, qr[i], adk[i]);
+                for (int i = 0; i < kDims; ++i) {
+                    adv[i].add(p * dr[i]);
+                    adk[i].add(ds * qr[i]);
                 }
             }
         }
     }
     if (!live) return;
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-        dk[rowoff + i] = adk[i] * scale;
-        dv[rowoff + i] = adv[i];
+    for (int i = 0; i < kDims; ++i) {
+        dk[rowoff + i] = adk[i].s * scale;
+        dv[rowoff + i] = adv[i].s;
     }
 }
 
@@ -259,7 +277,7 @@ static cudaError_t fwd_simt(const float *q, const float *k, const float *v, cons
     const size_t smem = 2 * 128 * D * sizeof(float);
     cudaFuncSetAttribute(k_fwd_simt<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     dim3 grid(m.T, Hq, m.B);
-    k_fwd_simt<D><<<grid, 128 * (D / 32), smem, s>>>(q, k, v, m, Hq, Hkv, scale, o, lse);
+    k_fwd_simt<D><<<grid, 128 * (D / kDims), smem, s>>>(q, k, v, m, Hq, Hkv, scale, o, lse);
     return cudaGetLastError();
 }
 
@@ -273,9 +291,9 @@ static cudaError_t bwd_simt(const float *q, const float *k, const float *v, cons
     const size_t smem = 2 * 128 * D * sizeof(float);
     cudaFuncSetAttribute(k_dq_simt<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     cudaFuncSetAttribute(k_dkdv_simt<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    k_dq_simt<D><<<dim3(m.T, Hq, m.B), 128 * (D / 32), smem, s>>>(q, k, v, dO, lse, Drow, m, Hq,
+    k_dq_simt<D><<<dim3(m.T, Hq, m.B), 128 * (D / kDims), smem, s>>>(q, k, v, dO, lse, Drow, m, Hq,
                                                                  Hkv, scale, dq);
-    k_dkdv_simt<D><<<dim3(m.T, Hkv, m.B), 128 * (D / 32), smem, s>>>(q, k, v, dO, lse, Drow, m, Hq,
+    k_dkdv_simt<D><<<dim3(m.T, Hkv, m.B), 128 * (D / kDims), smem, s>>>(q, k, v, dO, lse, Drow, m, Hq,
                                                                     Hkv, scale, dk, dv);
     return cudaGetLastError();
 }

@@ -12,6 +12,15 @@ namespace kvs {
 
 // ---------------------------------------------------------------- status word
 
+// Last CUDA runtime error seen by an entry point of this thread (see
+// kvs_last_cuda_error); cuda_status() records it and maps it to a status.
+extern thread_local const char *g_last_cuda_error;
+inline kvs_status cuda_status(cudaError_t e) {
+    if (e == cudaSuccess) return KVS_OK;
+    g_last_cuda_error = cudaGetErrorString(e);
+    return KVS_ERR_CUDA;
+}
+
 __device__ __forceinline__ void set_status(int32_t *st, int32_t code) {
     if (st) atomicCAS(st, 0, code);
 }

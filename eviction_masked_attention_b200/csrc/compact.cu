@@ -153,5 +153,5 @@ extern "C" kvs_status kvs_compact_block_table(int32_t *block_table, int32_t *blo
     k_compact<<<B, kCompactThreads, 0, s>>>(block_table, block_lpos, num_blocks, num_tokens,
                                            max_blocks, block_size, pool_blocks, ev, n_ev, freed,
                                            n_freed, dev_status);
-    return cudaGetLastError() == cudaSuccess ? KVS_OK : KVS_ERR_CUDA;
+    return cuda_status(cudaGetLastError());
 }

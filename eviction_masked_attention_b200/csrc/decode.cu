@@ -268,6 +268,12 @@ __global__ void __launch_bounds__(kDecWarps * 32)
     if (threadIdx.x == 0) counters[b * Hkv + kvh] = 0;
 }
 
+cudaError_t launch_decode_mma(int G, const void *q, const void *kc, const void *vc,
+                              const int32_t *bt, const int32_t *nt, int32_t B, int32_t Hq,
+                              int32_t Hkv, int32_t bs, int32_t max_blocks, float scale_log2,
+                              int32_t tps, int32_t max_splits, void *o, int32_t *counters,
+                              float *partials, int32_t *status, cudaStream_t s);
+
 struct DecodePlan {
     int32_t tps, max_splits;
     size_t counter_bytes, partial_bytes;
@@ -337,13 +343,12 @@ extern "C" kvs_status kvs_paged_decode_attn(const void *q, const void *k_cache, 
     launch_decode<T, DD, GG>(q, k_cache, v_cache, block_table, num_tokens, B, Hq, Hkv,           \
                              block_size, max_blocks, qs, p, o, ws, dev_status, s)
     if (bf) {
-        using bfh = __nv_bfloat16;
-        switch (G) {
-            case 1: KVS_DEC(bfh, 128, 1); break;
-            case 2: KVS_DEC(bfh, 128, 2); break;
-            case 4: KVS_DEC(bfh, 128, 4); break;
-            default: KVS_DEC(bfh, 128, 8); break;
-        }
+        // bf16: bulk-copy staging + warp-level tensor-core products
+        cudaError_t e = launch_decode_mma(G, q, k_cache, v_cache, block_table, num_tokens, B, Hq, Hkv,
+                                          block_size, max_blocks, qs, p.tps, p.max_splits, o,
+                                          (int32_t *)ws, (float *)((char *)ws + p.counter_bytes),
+                                          dev_status, s);
+        return cuda_status(e);
     } else {
         switch (G) {
             case 1: KVS_DEC(float, 64, 1); break;
@@ -353,5 +358,5 @@ extern "C" kvs_status kvs_paged_decode_attn(const void *q, const void *k_cache, 
         }
     }
 #undef KVS_DEC
-    return cudaGetLastError() == cudaSuccess ? KVS_OK : KVS_ERR_CUDA;
+    return cuda_status(cudaGetLastError());
 }

@@ -315,25 +315,26 @@ extern "C" kvs_status kvs_build_tile_mask(const kvs_evict_range *ev, int32_t n_e
     MaskWs w;
     mask_ws_layout(B, N, &w, (char *)ws);
     const int32_t BT = B * T;
-    if (cudaMemsetAsync(w.col_cnt, 0, sizeof(int32_t) * BT, s) != cudaSuccess) return KVS_ERR_CUDA;
-    if (cudaMemsetAsync(w.status, 0, sizeof(int32_t) * 4, s) != cudaSuccess) return KVS_ERR_CUDA;
-    if (cudaMemsetAsync(w.pairs, 0, sizeof(unsigned long long) * 2, s) != cudaSuccess)
-        return KVS_ERR_CUDA;
+    cudaError_t ce;
+    if ((ce = cudaMemsetAsync(w.col_cnt, 0, sizeof(int32_t) * BT, s)) != cudaSuccess ||
+        (ce = cudaMemsetAsync(w.status, 0, sizeof(int32_t) * 4, s)) != cudaSuccess ||
+        (ce = cudaMemsetAsync(w.pairs, 0, sizeof(unsigned long long) * 2, s)) != cudaSuccess)
+        return cuda_status(ce);
     if (n_ev > 0) k_validate_events<<<(n_ev + 255) / 256, 256, 0, s>>>(ev, n_ev, B, w.status);
     int64_t nthreads = (int64_t)B * N;
     k_kappa<<<(unsigned)((nthreads + 255) / 256), 256, 0, s>>>(ev, n_ev, B, N, m->kappa, w.pairs);
     k_classify<<<BT, 256, 0, s>>>(m->kappa, B, N, T, m->cls, w.row_nnz, w.row_npart, w.col_cnt);
     k_scan3<<<3, 1024, 0, s>>>(w.row_nnz, m->row_ptr, w.row_npart, w.row_poff, w.col_cnt,
                                m->col_ptr, BT);
-    if (cudaGetLastError() != cudaSuccess) return KVS_ERR_CUDA;
+    if ((ce = cudaGetLastError()) != cudaSuccess) return cuda_status(ce);
     int32_t h_nnz = 0, h_np = 0, h_st = 0;
     unsigned long long h_pairs = 0;
-    if (cudaMemcpyAsync(&h_nnz, m->row_ptr + BT, 4, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
-        cudaMemcpyAsync(&h_np, w.row_poff + BT, 4, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
-        cudaMemcpyAsync(&h_st, w.status, 4, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
-        cudaMemcpyAsync(&h_pairs, w.pairs, 8, cudaMemcpyDeviceToHost, s) != cudaSuccess)
-        return KVS_ERR_CUDA;
-    if (cudaStreamSynchronize(s) != cudaSuccess) return KVS_ERR_CUDA;
+    if ((ce = cudaMemcpyAsync(&h_nnz, m->row_ptr + BT, 4, cudaMemcpyDeviceToHost, s)) != cudaSuccess ||
+        (ce = cudaMemcpyAsync(&h_np, w.row_poff + BT, 4, cudaMemcpyDeviceToHost, s)) != cudaSuccess ||
+        (ce = cudaMemcpyAsync(&h_st, w.status, 4, cudaMemcpyDeviceToHost, s)) != cudaSuccess ||
+        (ce = cudaMemcpyAsync(&h_pairs, w.pairs, 8, cudaMemcpyDeviceToHost, s)) != cudaSuccess)
+        return cuda_status(ce);
+    if ((ce = cudaStreamSynchronize(s)) != cudaSuccess) return cuda_status(ce);
     if (h_st != 0) return (kvs_status)h_st;
     sizes->nnz = h_nnz;
     sizes->n_partial = h_np;
@@ -348,6 +349,6 @@ extern "C" kvs_status kvs_build_tile_mask(const kvs_evict_range *ev, int32_t n_e
         m->bits);
     k_fill_cols<<<(BT + rows_per_cta - 1) / rows_per_cta, 32 * rows_per_cta, 0, s>>>(
         m->cls, B, T, m->col_ptr, w.tile_pidx, m->col_row, m->col_pidx);
-    if (cudaGetLastError() != cudaSuccess) return KVS_ERR_CUDA;
+    if ((ce = cudaGetLastError()) != cudaSuccess) return cuda_status(ce);
     return KVS_OK;
 }

@@ -152,5 +152,5 @@ extern "C" kvs_status kvs_rope_logical(const void *x, int64_t x_tok_stride, void
                                                       (const bf *)v, v_tok_stride, (bf *)v_out,
                                                       dev_status);
     }
-    return cudaGetLastError() == cudaSuccess ? KVS_OK : KVS_ERR_CUDA;
+    return cuda_status(cudaGetLastError());
 }

@@ -201,13 +201,18 @@ kvs_status kvs_paged_decode_attn(const void *q, const void *k_cache, const void 
  *   lse_t = ln sum_{j visible} exp(scale <q_t, k_j>)
  * using the compiled mask m (EMPTY tiles skipped, PARTIAL tiles bit-masked).
  *   q, o    [B][N][Hq][d];  k, v [B][N][Hkv][d];  lse fp32 [B][Hq][N]
+ *   o_lo    optional (NULL to skip), bf16 only, same layout as o: the rounding
+ *           residual bf16(O - o) of the bf16 output, so that o + o_lo carries
+ *           about 16 significant bits of the fp32 result. Pass it to the
+ *           backward, which then forms D_t = <dO_t, O_t> from o + o_lo instead
+ *           of the rounded o (the dominant bf16 error of the gradients).
  *   dt      KVS_BF16 (d = 128; tcgen05 tensor cores, fp32 accumulation) or
  *           KVS_F32 (d in {64, 128}; fp32 CUDA cores)
  * Pointers of bf16 tensors must be 16-byte aligned.
  */
 kvs_status kvs_masked_attn_fwd(const void *q, const void *k, const void *v, const kvs_tile_mask *m,
                                int32_t B, int32_t N, int32_t Hq, int32_t Hkv, int32_t d,
-                               float scale, kvs_dtype dt, void *o, float *lse,
+                               float scale, kvs_dtype dt, void *o, void *o_lo, float *lse,
                                int32_t *dev_status, kvs_stream_t stream);
 
 /*
@@ -217,15 +222,29 @@ kvs_status kvs_masked_attn_fwd(const void *q, const void *k, const void *v, cons
  *   dQ_t = scale sum_j dS_tj k_j;  dK_j = scale sum_t dS_tj q_t;
  * dK, dV of a kv head sum over its Hq/Hkv query heads.
  *   o, dO, dq [B][N][Hq][d]; dk, dv [B][N][Hkv][d]; lse as returned by the forward.
+ *   o_lo    optional residual written by the forward (NULL: D uses o alone).
  *   ws      device scratch of kvs_masked_attn_bwd_ws_bytes(...) bytes.
+ *   stages  bitmask of the three kernels the backward consists of:
+ *           KVS_BWD_PREP (D and lse rows into ws), KVS_BWD_DKDV, KVS_BWD_DQ;
+ *           KVS_BWD_ALL runs all three in order. Running them in separate calls
+ *           (same ws, PREP first) gives the same result; dq is only written by
+ *           KVS_BWD_DQ, dk and dv only by KVS_BWD_DKDV. The fp32 path ignores
+ *           the mask and always runs everything.
+ * Results are deterministic (no atomics).
  */
+enum { KVS_BWD_PREP = 1, KVS_BWD_DKDV = 2, KVS_BWD_DQ = 4, KVS_BWD_ALL = 7 };
 size_t kvs_masked_attn_bwd_ws_bytes(int32_t B, int32_t N, int32_t Hq, int32_t Hkv, int32_t d,
                                     kvs_dtype dt);
 kvs_status kvs_masked_attn_bwd(const void *q, const void *k, const void *v, const void *o,
-                               const void *dO, const float *lse, const kvs_tile_mask *m, int32_t B,
+                               const void *o_lo, const void *dO, const float *lse, const kvs_tile_mask *m, int32_t B,
                                int32_t N, int32_t Hq, int32_t Hkv, int32_t d, float scale,
                                kvs_dtype dt, void *dq, void *dk, void *dv, void *ws,
-                               size_t ws_bytes, int32_t *dev_status, kvs_stream_t stream);
+                               size_t ws_bytes, int32_t stages, int32_t *dev_status,
+                               kvs_stream_t stream);
+
+/* Text of the last CUDA runtime error behind a KVS_ERR_CUDA returned to the
+ * calling thread ("no error" if there was none); a static string. */
+const char *kvs_last_cuda_error(void);
 
 /* Human-readable name of a status code (static string). */
 const char *kvs_status_str(kvs_status s);

@@ -53,7 +53,7 @@ def test_host_side_argument_errors(built):
     m = kvs._TileMaskC()
     m.B, m.N, m.T = 1, 100, 1
     assert L.kvs_masked_attn_fwd(None, None, None, ctypes.byref(m), 1, 100, 4, 1, 96, 1.0, kvs.KVS_BF16,
-                                 None, None, None, None) == kvs.KVS_ERR_INVALID_ARG
+                                 None, None, None, None, None) == kvs.KVS_ERR_INVALID_ARG
 
 
 def test_product_path_has_no_oracle_import():

@@ -17,10 +17,11 @@ def _run(cfg, ev, q, k, v, do, bwd=True):
     gm = kvs.kvs_build_tile_mask(events_dev(ev), cfg.batch, cfg.n_tokens)
     qd, kd, vd = dev(q, tdt), dev(k, tdt), dev(v, tdt)
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
-    o, lse = kvs.kvs_masked_attn_fwd(qd, kd, vd, gm, cfg.scale, status=status)
+    o, lse, o_lo = kvs.kvs_masked_attn_fwd(qd, kd, vd, gm, cfg.scale, status=status)
     out = dict(o=o, lse=lse, mask=gm)
     if bwd:
-        dq, dk, dv = kvs.kvs_masked_attn_bwd(qd, kd, vd, o, dev(do, tdt), lse, gm, cfg.scale, status=status)
+        dq, dk, dv = kvs.kvs_masked_attn_bwd(qd, kd, vd, o, dev(do, tdt), lse, gm, cfg.scale, status=status,
+                                             o_lo=o_lo)
         out.update(dq=dq, dk=dk, dv=dv)
     torch.cuda.synchronize()
     assert status.item() == 0, kvs.status_str(status.item())
@@ -40,7 +41,8 @@ def _check_full(cfg, ev, q, k, v, do, tol, bwd=True):
         for name, want in (("dq", dq), ("dk", dk), ("dv", dv)):
             got = host(r[name])
             assert_close(got, want, tol, name)
-            assert rel_l2(got, want) <= GRAD_REL_L2, (name, rel_l2(got, want))
+            rl = rel_l2(got, want)
+            assert rl is None or rl <= GRAD_REL_L2, (name, rl)
     return r
 
 
@@ -92,7 +94,7 @@ def test_bf16_rope_then_attention_end_to_end():
     qd = kvs.kvs_rope_logical(dev(q[0], torch.bfloat16), dev(lp), cfg.theta)[None]
     kd = kvs.kvs_rope_logical(dev(k[0], torch.bfloat16), dev(lp), cfg.theta)[None]
     gm = kvs.kvs_build_tile_mask(events_dev(ev), 1, N)
-    o, lse = kvs.kvs_masked_attn_fwd(qd.contiguous(), kd.contiguous(), dev(v, torch.bfloat16), gm, cfg.scale)
+    o, lse, _ = kvs.kvs_masked_attn_fwd(qd.contiguous(), kd.contiguous(), dev(v, torch.bfloat16), gm, cfg.scale)
     kap = oracle.kappa(ev, 1, N)
     qo = oracle.rope(q[0], lp, cfg.theta)[None]
     ko = oracle.rope(k[0], lp, cfg.theta)[None]
@@ -118,10 +120,10 @@ def test_full_size_sampled(cid):
     q, k, v, do = W.replay_tensors_device(cfg)
     gm = kvs.kvs_build_tile_mask(events_dev(ev), B, N)
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
-    o, lse = kvs.kvs_masked_attn_fwd(q, k, v, gm, cfg.scale, status=status)
+    o, lse, o_lo = kvs.kvs_masked_attn_fwd(q, k, v, gm, cfg.scale, status=status)
     bwd = cid in (3, 5)
     if bwd:
-        dq, dk, dv = kvs.kvs_masked_attn_bwd(q, k, v, o, do, lse, gm, cfg.scale, status=status)
+        dq, dk, dv = kvs.kvs_masked_attn_bwd(q, k, v, o, do, lse, gm, cfg.scale, status=status, o_lo=o_lo)
     torch.cuda.synchronize()
     assert status.item() == 0
     kap = oracle.kappa(ev, B, N)
@@ -145,12 +147,23 @@ def test_full_size_sampled(cid):
                 assert_close(host(dk[b, cols, kvh]), wk, BF16_TOL, f"dK b{b}")
                 assert_close(host(dv[b, cols, kvh]), wv, BF16_TOL, f"dV b{b}")
     if bwd:
-        # properties at full size: sum_j dK_j = 0 and sum_j dV_j = sum over the group of dO_t
-        # (rows of P sum to 1; rows of dS sum to dO.(O - bf16(O)), a rounding-size term)
+        # properties at full size, exact for the true gradients:
+        #   sum_j dV_j = sum over the group of dO_t   (every row of P sums to 1)
+        #   sum_j dK_j = 0                            (every row of dS sums to 0)
+        # The stored gradients are bf16, so each element may be off by half an
+        # ulp (2^-9 |x|); and D_t = <dO_t, O_t> is formed from o + o_lo, whose
+        # error moves row sums of dS by at most 2^-17 sum_i |dO_ti O_ti|.
+        # The bounds below add those rounding terms up (worst case) plus 0.05.
+        r9 = 2.0 ** -9
         for b in (0, B - 1):
-            sdk = dk[b].double().sum(0)                        # [Hkv, d]
-            sdv = dv[b].double().sum(0)
-            sdo = do[b].double().sum(0).view(Hkv, G, -1).sum(1)
-            ek, ev_ = sdk.abs().max().item(), (sdv - sdo).abs().max().item()
-            print(f"cfg{cid} b{b}: |sum dK| {ek:.3g}, |sum dV - sum dO| {ev_:.3g}, |sum dO| {sdo.abs().max().item():.3g}")
-            assert ek <= 5.0 and ev_ <= 1.0
+            dkb, dvb, dob = dk[b].double(), dv[b].double(), do[b].double()
+            sdv = dvb.sum(0)                                     # [Hkv, d]
+            sdo = dob.sum(0).view(Hkv, G, -1).sum(1)
+            tol_v = r9 * dvb.abs().sum(0) + 0.05
+            assert ((sdv - sdo).abs() <= tol_v).all(), float((sdv - sdo).abs().max())
+            ob, qb = o[b].double(), q[b].double()                # [N, Hq, d]
+            dmax = (2.0 ** -17 * (dob * ob).abs().sum(-1))       # [N, Hq] bound on |dS row sum|
+            qterm = (dmax[..., None] * qb.abs()).view(N, Hkv, G, -1).sum((0, 2)) * cfg.scale
+            tol_k = r9 * dkb.abs().sum(0) + qterm + 0.05
+            sdk = dkb.sum(0)
+            assert (sdk.abs() <= tol_k).all(), float(sdk.abs().max())
