@@ -32,7 +32,7 @@ EXPORTED = (
     "kvs_build_tile_mask_ws_bytes", "kvs_build_tile_mask", "kvs_compact_block_table",
     "kvs_rope_logical", "kvs_paged_decode_ws_bytes", "kvs_paged_decode_attn",
     "kvs_masked_attn_fwd", "kvs_masked_attn_bwd_ws_bytes", "kvs_masked_attn_bwd",
-    "kvs_status_str", "kvs_version", "kvs_last_cuda_error",
+    "kvs_status_str", "kvs_version", "kvs_last_cuda_error", "kvs_paged_decode_attn_static",
 )
 
 

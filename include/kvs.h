@@ -195,6 +195,32 @@ kvs_status kvs_paged_decode_attn(const void *q, const void *k_cache, const void 
                                  size_t ws_bytes, int32_t *dev_status, kvs_stream_t stream);
 
 /*
+ * kvs_paged_decode_attn for callers that cannot allocate device memory.
+ * The pages have no counterpart to this call; it exists for users whose decode
+ * path must not call cudaMalloc (CUDA-graph replay of generation steps, engines
+ * whose pool allocator owns all device memory, embedders that only receive
+ * input/output pointers). Same arguments and results as kvs_paged_decode_attn
+ * minus ws/ws_bytes: the scratch is a fixed array of
+ * KVS_DECODE_STATIC_SCRATCH_BYTES (16 MiB) compiled into the library, held in
+ * the memory of every GPU that loads it until the process exits.
+ *  - Returns KVS_ERR_CAPACITY (nothing launched) when the call needs more
+ *    scratch than that, i.e. kvs_paged_decode_ws_bytes(...) > the maximum.
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress), zeroes it and synchronizes the device; make that
+ *    first call before any stream capture.
+ *  - All calls share the array: calls whose kernels overlap on the GPU
+ *    (unordered streams, concurrent threads) race and give wrong results.
+ *  - Allocates nothing: no cudaMalloc/cudaFree, no allocating library call.
+ */
+#define KVS_DECODE_STATIC_SCRATCH_BYTES ((size_t)16 << 20)
+kvs_status kvs_paged_decode_attn_static(const void *q, const void *k_cache, const void *v_cache,
+                                        const int32_t *block_table, const int32_t *num_tokens,
+                                        int32_t B, int32_t Hq, int32_t Hkv, int32_t d,
+                                        int32_t block_size, int32_t max_blocks, float scale,
+                                        kvs_dtype dt, void *o, int32_t *dev_status,
+                                        kvs_stream_t stream);
+
+/*
  * Eviction-masked causal attention forward over the continuous trace ([T]
  * trainer replay; [P] Fig. 2(A)):
  *   O_t = sum_{j visible from t} softmax_j(scale <q_t, k_j>) v_j,
