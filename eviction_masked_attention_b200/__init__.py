@@ -244,8 +244,7 @@ def kvs_rope_logical(x, lpos, theta: float, inverse: bool = False, out=None, out
 
 def kvs_paged_decode_attn(q, k_cache, v_cache, block_table, num_tokens, block_size: int, scale: float,
                           out=None, ws=None, status=None):
-    """q [B, Hq, d]; caches [pool, Hkv, bs, d]; returns o [B, Hq, d].
-    ``ws`` (uint8) must be zeroed before its first use; the call leaves it reusable."""
+    """q [B, Hq, d]; caches [pool, Hkv, bs, d]; returns o [B, Hq, d]."""
     _dev(q, k_cache, v_cache, block_table, num_tokens)
     B, Hq, d = q.shape
     Hkv = k_cache.shape[1]
@@ -253,7 +252,7 @@ def kvs_paged_decode_attn(q, k_cache, v_cache, block_table, num_tokens, block_si
     L = lib()
     wsb = L.kvs_paged_decode_ws_bytes(B, Hq, Hkv, d, block_size, M)
     if ws is None:
-        ws = torch.zeros(wsb, dtype=torch.uint8, device=q.device)
+        ws = torch.empty(wsb, dtype=torch.uint8, device=q.device)
     if out is None:
         out = torch.empty_like(q)
     if status is None:

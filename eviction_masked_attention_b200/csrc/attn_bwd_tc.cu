@@ -103,6 +103,7 @@ struct DkvSmem {
     uint8_t dout[2][kTile];
     float l2[2][128];
     float dd[2][128];
+    int32_t q0[2], full_tile[2];  // query tile origin and FULL flag of the item in each stage
     uint64_t kv_full, full[2], empty[2], st_full, dp_full, p_ready, ds_ready, acc_done, fin;
     uint32_t tmem_base;
     int abort;
@@ -167,6 +168,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 if (n >= 2 && !mbar_wait(&S.empty[s], ((n >> 1) - 1) & 1, abort, status)) break;
                 const int e = n / G, g = n % G, h = kvh * G + g;
                 const int q0 = m.col_row[c0 + e] * 128;
+                S.q0[s] = q0;
+                S.full_tile[s] = m.col_pidx[c0 + e] < 0;
                 mbar_expect_tx(&S.full[s], 2 * kTile + 1024);
                 tma_load_4d(S.q[s], &tmQ, &S.full[s], 0, h, q0, b);
                 tma_load_4d(S.q[s] + kTile / 2, &tmQ, &S.full[s], 64, h, q0, b);
@@ -231,9 +234,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         bool ok = true;
         for (int n = 0; n < nw; ++n) {
             const int s = n & 1;
-            const int e = n / G;
-            const int q0 = m.col_row[c0 + e] * 128;
-            const bool full = m.col_pidx[c0 + e] < 0;
+            if (!warp_wait(&S.full[s], (n >> 1) & 1, abort, status)) {
+                ok = false;
+                break;
+            }
+            const int q0 = S.q0[s];
+            const bool full = S.full_tile[s] != 0;
             // visible query rows of this key inside the tile: [rlo, rhi) (j <= t < kappa_j)
             int rlo = 0, rhi = 128;
             if (!full) {
@@ -247,8 +253,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             }
             rlo -= col0;
             rhi -= col0;
-            if (!warp_wait(&S.full[s], (n >> 1) & 1, abort, status) ||
-                !warp_wait(&S.st_full, n & 1, abort, status)) {
+            if (!warp_wait(&S.st_full, n & 1, abort, status)) {
                 ok = false;
                 break;
             }
@@ -350,6 +355,8 @@ struct DqSmem {
     uint8_t dout[kTile];
     uint8_t k[2][kTile];
     uint8_t v[2][kTile];
+    uint32_t bits[2][128 * 4];  // mask rows of the key tile in each stage (partial tiles)
+    int32_t pid[2];             // its partial index (-1: full)
     uint64_t qo_full, full[2], empty[2], s_full, dp_full, s_free, dp_free, ds_ready, dq_done,
         acc_done, fin;
     uint32_t tmem_base;
@@ -414,11 +421,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 const int s = n & 1;
                 if (n >= 2 && !mbar_wait(&S.empty[s], ((n >> 1) - 1) & 1, abort, status)) break;
                 const int k0 = m.row_col[e0 + n] * 128;
-                mbar_expect_tx(&S.full[s], 2 * kTile);
+                const int32_t pid = m.row_pidx[e0 + n];
+                S.pid[s] = pid;
+                mbar_expect_tx(&S.full[s], 2 * kTile + (pid >= 0 ? 2048u : 0u));
                 tma_load_4d(S.k[s], &tmK, &S.full[s], 0, kvh, k0, b);
                 tma_load_4d(S.k[s] + kTile / 2, &tmK, &S.full[s], 64, kvh, k0, b);
                 tma_load_4d(S.v[s], &tmV, &S.full[s], 0, kvh, k0, b);
                 tma_load_4d(S.v[s] + kTile / 2, &tmV, &S.full[s], 64, kvh, k0, b);
+                if (pid >= 0) bulk_load(S.bits[s], m.bits + (int64_t)pid * 512, 2048, &S.full[s]);
             }
         }
     } else if (warp == 1) {
@@ -480,15 +490,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         bool ok = true;
         for (int n = 0; n < nt; ++n) {
             const int s = n & 1;
-            const int32_t pid = m.row_pidx[e0 + n];
-            uint2 bits = make_uint2(~0u, ~0u);
-            if (pid >= 0)
-                bits = *reinterpret_cast<const uint2 *>(m.bits + (int64_t)pid * 512 + row * 4 + half * 2);
             if (!warp_wait(&S.s_full, n & 1, abort, status)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
+            // S_n complete implies stage s (K, V and the tile's mask rows) has
+            // landed; it is refilled only after dQ_n, i.e. after this item's dS
+            uint2 bits = make_uint2(~0u, ~0u);
+            if (S.pid[s] >= 0) bits = *reinterpret_cast<const uint2 *>(&S.bits[s][row * 4 + half * 2]);
             float p[64];
             {
                 uint32_t r0[32], r1[32];

@@ -284,6 +284,8 @@ struct Fwd2Smem {
     uint8_t q[2][kTileBytes];
     uint8_t k[2][kTileBytes];
     uint8_t v[2][kTileBytes];
+    uint32_t bits[2][128 * 4];  // mask rows of the tile in each V stage (partial tiles)
+    int32_t pid[2];             // partial index of the tile in each V stage (-1: full)
     uint64_t bar_q, kfull[2], kempty[2], vfull[2], vempty[2], sfull[2], pfull[2], odone[2], fin;
     uint32_t tmem_base;
     int abort;
@@ -351,9 +353,14 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
                 tma_load_4d(S.k[s], &tmK, &S.kfull[s], 0, kvh, k0, b);
                 tma_load_4d(S.k[s] + kTileBytes / 2, &tmK, &S.kfull[s], 64, kvh, k0, b);
                 if (n >= 2 && !mbar_wait(&S.vempty[s], ph, abort, status)) break;
-                mbar_expect_tx(&S.vfull[s], kTileBytes);
+                // the tile's mask metadata travels with its V stage, which is only
+                // released after both heads' softmax finished this tile
+                const int32_t pid = m.row_pidx[e0 + n];
+                S.pid[s] = pid;
+                mbar_expect_tx(&S.vfull[s], kTileBytes + (pid >= 0 ? 2048u : 0u));
                 tma_load_4d(S.v[s], &tmV, &S.vfull[s], 0, kvh, k0, b);
                 tma_load_4d(S.v[s] + kTileBytes / 2, &tmV, &S.vfull[s], 64, kvh, k0, b);
+                if (pid >= 0) bulk_load(S.bits[s], m.bits + (int64_t)pid * 512, 2048, &S.vfull[s]);
             }
         }
     } else if (warp == 1) {
@@ -422,15 +429,17 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
         float m_run = -INFINITY, l_run = 0.f;
         bool ok = true;
         for (int n = 0; n < nt; ++n) {
-            const int32_t pid = m.row_pidx[e0 + n];
-            uint4 bits = make_uint4(~0u, ~0u, ~0u, ~0u);
-            if (pid >= 0)
-                bits = *reinterpret_cast<const uint4 *>(m.bits + (int64_t)pid * 512 + row * 4);
             if (!__all_sync(0xffffffffu, mbar_wait(&S.sfull[x], n & 1, abort, status))) {
                 ok = false;
                 break;
             }
+            if (!__all_sync(0xffffffffu, mbar_wait(&S.vfull[n & 1], (n >> 1) & 1, abort, status))) {
+                ok = false;
+                break;
+            }
             tc_fence_after();
+            uint4 bits = make_uint4(~0u, ~0u, ~0u, ~0u);
+            if (S.pid[n & 1] >= 0) bits = *reinterpret_cast<const uint4 *>(&S.bits[n & 1][row * 4]);
             const uint32_t wb[4] = {bits.x, bits.y, bits.z, bits.w};
             // pass 1: row maximum of the masked, base-2 scaled scores
             float mt = -INFINITY;

@@ -12,8 +12,7 @@
 // queries held in shared memory, the warp runs an online softmax (base-2,
 // pre-scaled logits), and lanes (16 per row, 2 rows at a time) accumulate
 // 16-byte slices of the value rows. Warp states merge in shared memory; with
-// several splits, the last CTA of a (sequence, kv head) to finish merges the
-// split partials (a counter per unit, returned to zero by that CTA).
+// several splits, each CTA writes its partial and k_decode_combine merges them.
 #include <algorithm>
 
 #include "common.cuh"
@@ -46,14 +45,13 @@ __device__ __forceinline__ void store_out(__nv_bfloat16 *o, int i, float v) {
     o[i] = __float2bfloat16_rn(v);
 }
 
-// ws: [unit counters: B*Hkv int32, padded to 256 B][partials: B*Hq*S*(D+2) fp32]
+// ws: partials [B][Hq][max_splits][D + 2] fp32 (unnormalised output, max, sum)
 template <typename T, int D, int G>
 __global__ void __launch_bounds__(kDecWarps * 32)
     k_decode(const T *__restrict__ q, const T *__restrict__ kc, const T *__restrict__ vc,
              const int32_t *__restrict__ block_table, const int32_t *__restrict__ num_tokens,
              int32_t Hq, int32_t Hkv, int32_t bs, int32_t max_blocks, float qscale, int32_t tps,
-             int32_t max_splits, T *__restrict__ o, int32_t *counters, float *partials,
-             int32_t *status) {
+             int32_t max_splits, T *__restrict__ o, float *partials, int32_t *status) {
     using R = Row16<T>;
     constexpr int E = R::E;           // elements per 16 bytes
     static_assert(D * sizeof(T) == 256, "rows are 256 bytes");
@@ -68,7 +66,6 @@ __global__ void __launch_bounds__(kDecWarps * 32)
     __shared__ __align__(16) float s_p[kDecWarps][16][G];
     __shared__ float s_m[kDecWarps][G], s_l[kDecWarps][G];
     __shared__ __align__(16) float s_acc[kDecWarps][G][D];
-    __shared__ int s_last;
 
     for (int i = threadIdx.x; i < G * D; i += blockDim.x) {
         const int g = i / D, e = i % D;
@@ -240,56 +237,58 @@ __global__ void __launch_bounds__(kDecWarps * 32)
             }
         }
     }
-    if (single) return;
-    __threadfence();
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        const int prev = atomicAdd(&counters[b * Hkv + kvh], 1);
-        s_last = prev == nsplit - 1;
-    }
-    __syncthreads();
-    if (!s_last) return;
-    __threadfence();
-    for (int i = threadIdx.x; i < G * D; i += blockDim.x) {
-        const int g = i / D, e = i % D;
-        const float *pg = part + (int64_t)g * max_splits * (D + 2);
-        float M = -INFINITY;
-        for (int sp = 0; sp < nsplit; ++sp) M = fmaxf(M, __ldcg(pg + sp * (D + 2) + D));
-        const float Mr = M == -INFINITY ? 0.f : M;
-        float L = 0.f, A = 0.f;
-        for (int sp = 0; sp < nsplit; ++sp) {
-            const float *pp = pg + sp * (D + 2);
-            const float f = ex2(__ldcg(pp + D) - Mr);
-            L += __ldcg(pp + D + 1) * f;
-            A += __ldcg(pp + e) * f;
-        }
-        store_out(o, ((int)((int64_t)b * Hq + kvh * G + g)) * D + e, L > 0.f ? A / L : 0.f);
-    }
-    if (threadIdx.x == 0) counters[b * Hkv + kvh] = 0;
 }
 
 cudaError_t launch_decode_mma(int G, const void *q, const void *kc, const void *vc,
                               const int32_t *bt, const int32_t *nt, int32_t B, int32_t Hq,
                               int32_t Hkv, int32_t bs, int32_t max_blocks, float scale_log2,
-                              int32_t tps, int32_t max_splits, void *o, int32_t *counters,
-                              float *partials, int32_t *status, cudaStream_t s);
+                              int32_t tps, int32_t max_splits, void *o, float *partials,
+                              int32_t *status, cudaStream_t s);
+
+// Merge the split partials of one (sequence, query head): thread e owns output
+// dim e; every split's (max, sum) pair is read by all threads (broadcast).
+template <typename T, int D>
+__global__ void __launch_bounds__(D)
+    k_decode_combine(const int32_t *__restrict__ num_tokens, int32_t Hq, int32_t bs,
+                     int32_t max_blocks, int32_t tps, int32_t max_splits,
+                     const float *__restrict__ partials, T *__restrict__ o) {
+    const int h = blockIdx.x, b = blockIdx.y, e = threadIdx.x;
+    const int32_t ntok = min(max(num_tokens[b], 0), max_blocks * bs);
+    const int32_t nsplit = max(1, (ntok + tps - 1) / tps);
+    if (nsplit == 1) return;  // the split kernel wrote the output itself
+    const float *pg = partials + ((int64_t)b * Hq + h) * max_splits * (D + 2);
+    float M = -INFINITY;
+#pragma unroll 8
+    for (int sp = 0; sp < nsplit; ++sp) M = fmaxf(M, pg[sp * (D + 2) + D]);
+    const float Mr = M == -INFINITY ? 0.f : M;
+    float L = 0.f, A = 0.f;
+#pragma unroll 8
+    for (int sp = 0; sp < nsplit; ++sp) {
+        const float *pp = pg + sp * (D + 2);
+        const float f = ex2(pp[D] - Mr);
+        L += pp[D + 1] * f;
+        A += pp[e] * f;
+    }
+    store_out(o, (int)(((int64_t)b * Hq + h) * D + e), L > 0.f ? A / L : 0.f);
+}
 
 struct DecodePlan {
     int32_t tps, max_splits;
-    size_t counter_bytes, partial_bytes;
+    size_t partial_bytes;
 };
 
+// Entries per split: as many as keep at least two waves of CTAs busy on 148 SMs
+// when sequences are half full, between 128 and 1024.
 inline DecodePlan decode_plan(int32_t B, int32_t Hq, int32_t Hkv, int32_t d, int32_t bs,
                               int32_t max_blocks) {
     DecodePlan p;
     const int64_t max_tok = (int64_t)max_blocks * bs;
     const int64_t units = (int64_t)B * Hkv;
     int32_t tps = 1024;
-    while (tps > 256 && units * ((max_tok / 2 + tps - 1) / tps) < 148 * 4) tps >>= 1;
+    while (tps > 128 && units * ((max_tok / 2 + tps - 1) / tps) < 148 * 8) tps >>= 1;
     p.tps = tps;
     p.max_splits = (int32_t)std::max<int64_t>(1, (max_tok + tps - 1) / tps);
-    p.counter_bytes = (((size_t)B * Hkv * sizeof(int32_t)) + 255) & ~(size_t)255;
-    p.partial_bytes = (size_t)B * Hq * p.max_splits * (d + 2) * sizeof(float);
+    p.partial_bytes = p.max_splits > 1 ? (size_t)B * Hq * p.max_splits * (d + 2) * sizeof(float) : 16;
     return p;
 }
 
@@ -299,11 +298,9 @@ void launch_decode(const void *q, const void *kc, const void *vc, const int32_t 
                    int32_t max_blocks, float qscale, const DecodePlan &p, void *o, void *ws,
                    int32_t *status, cudaStream_t s) {
     dim3 grid(p.max_splits, Hkv, B);
-    int32_t *counters = (int32_t *)ws;
-    float *partials = (float *)((char *)ws + p.counter_bytes);
     k_decode<T, D, G><<<grid, kDecWarps * 32, 0, s>>>(
         (const T *)q, (const T *)kc, (const T *)vc, bt, nt, Hq, Hkv, bs, max_blocks, qscale, p.tps,
-        p.max_splits, (T *)o, counters, partials, status);
+        p.max_splits, (T *)o, (float *)ws, status);
 }
 
 }  // namespace kvs
@@ -313,8 +310,7 @@ using namespace kvs;
 extern "C" size_t kvs_paged_decode_ws_bytes(int32_t B, int32_t Hq, int32_t Hkv, int32_t d,
                                             int32_t block_size, int32_t max_blocks) {
     if (B <= 0 || Hq <= 0 || Hkv <= 0 || d <= 0 || block_size <= 0 || max_blocks <= 0) return 0;
-    DecodePlan p = decode_plan(B, Hq, Hkv, d, block_size, max_blocks);
-    return p.counter_bytes + p.partial_bytes;
+    return decode_plan(B, Hq, Hkv, d, block_size, max_blocks).partial_bytes;
 }
 
 extern "C" kvs_status kvs_paged_decode_attn(const void *q, const void *k_cache, const void *v_cache,
@@ -335,28 +331,36 @@ extern "C" kvs_status kvs_paged_decode_attn(const void *q, const void *k_cache, 
     const bool bf = dt == KVS_BF16 && d == 128, f32 = dt == KVS_F32 && d == 64;
     if (!bf && !f32) return KVS_ERR_UNSUPPORTED;
     if (G != 1 && G != 2 && G != 4 && G != 8) return KVS_ERR_UNSUPPORTED;
-    DecodePlan p = decode_plan(B, Hq, Hkv, d, block_size, max_blocks);
-    if (ws_bytes < p.counter_bytes + p.partial_bytes) return KVS_ERR_CAPACITY;
+    const DecodePlan p = decode_plan(B, Hq, Hkv, d, block_size, max_blocks);
+    if (ws_bytes < p.partial_bytes) return KVS_ERR_CAPACITY;
     const float qs = scale * 1.4426950408889634f;  // base-2 logits
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-#define KVS_DEC(T, DD, GG)                                                                      \
-    launch_decode<T, DD, GG>(q, k_cache, v_cache, block_table, num_tokens, B, Hq, Hkv,           \
-                             block_size, max_blocks, qs, p, o, ws, dev_status, s)
+    cudaError_t e = cudaSuccess;
     if (bf) {
         // bf16: bulk-copy staging + warp-level tensor-core products
-        cudaError_t e = launch_decode_mma(G, q, k_cache, v_cache, block_table, num_tokens, B, Hq, Hkv,
-                                          block_size, max_blocks, qs, p.tps, p.max_splits, o,
-                                          (int32_t *)ws, (float *)((char *)ws + p.counter_bytes),
-                                          dev_status, s);
-        return cuda_status(e);
+        e = launch_decode_mma(G, q, k_cache, v_cache, block_table, num_tokens, B, Hq, Hkv,
+                              block_size, max_blocks, qs, p.tps, p.max_splits, o, (float *)ws,
+                              dev_status, s);
+        if (e != cudaSuccess) return cuda_status(e);
+        if (p.max_splits > 1)
+            k_decode_combine<__nv_bfloat16, 128><<<dim3(Hq, B), 128, 0, s>>>(
+                num_tokens, Hq, block_size, max_blocks, p.tps, p.max_splits, (const float *)ws,
+                (__nv_bfloat16 *)o);
     } else {
+#define KVS_DEC(GG)                                                                              \
+    launch_decode<float, 64, GG>(q, k_cache, v_cache, block_table, num_tokens, B, Hq, Hkv,       \
+                                 block_size, max_blocks, qs, p, o, ws, dev_status, s)
         switch (G) {
-            case 1: KVS_DEC(float, 64, 1); break;
-            case 2: KVS_DEC(float, 64, 2); break;
-            case 4: KVS_DEC(float, 64, 4); break;
-            default: KVS_DEC(float, 64, 8); break;
+            case 1: KVS_DEC(1); break;
+            case 2: KVS_DEC(2); break;
+            case 4: KVS_DEC(4); break;
+            default: KVS_DEC(8); break;
         }
-    }
 #undef KVS_DEC
+        if (p.max_splits > 1)
+            k_decode_combine<float, 64><<<dim3(Hq, B), 64, 0, s>>>(
+                num_tokens, Hq, block_size, max_blocks, p.tps, p.max_splits, (const float *)ws,
+                (float *)o);
+    }
     return cuda_status(cudaGetLastError());
 }

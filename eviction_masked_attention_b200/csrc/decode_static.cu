@@ -6,8 +6,7 @@
 // while a step runs, and embedders that only get device pointers for inputs
 // and outputs. For them, kvs_paged_decode_attn_static runs the same split-K
 // decode as kvs_paged_decode_attn but takes its scratch (the per-split softmax
-// partials and the per-(sequence, kv head) merge counters) from one fixed
-// array compiled into this file.
+// partials) from one fixed array compiled into this file.
 //
 // The array lives in device global memory of every GPU that loads this part
 // of the library, for the life of the process. Its size is the stated maximum
@@ -16,11 +15,10 @@
 //
 // In host code the array's name does not stand for a device address (it is a
 // host-side shadow symbol). The device address is obtained once per device,
-// with that device current, through cudaGetSymbolAddress; the same first call
-// zeroes the array (the merge counters must start at zero; each call leaves
-// them at zero again) and waits for that to finish. That set-up happens inside
-// the first call on each device, so the first call must not be made while a
-// stream is being captured.
+// with that device current, through cudaGetSymbolAddress. That set-up happens
+// inside the first call on each device, so the first call must not be made
+// while a stream is being captured. Nothing in the array has to start at zero:
+// every call writes the partials it later reads.
 //
 // All calls share the one array: two calls whose kernels overlap on the GPU
 // (different streams without ordering, or concurrent host threads) race on it
@@ -50,10 +48,6 @@ kvs_status scratch_on_current_device(void **out) {
         e = cudaGetSymbolAddress(&p, g_decode_scratch);
         if (e != cudaSuccess) return cuda_status(e);
         if (!p) return KVS_ERR_CUDA;
-        e = cudaMemset(p, 0, KVS_DECODE_STATIC_SCRATCH_BYTES);
-        if (e != cudaSuccess) return cuda_status(e);
-        e = cudaDeviceSynchronize();
-        if (e != cudaSuccess) return cuda_status(e);
         g_scratch_addr[dev] = p;
     }
     *out = g_scratch_addr[dev];

@@ -181,9 +181,10 @@ kvs_status kvs_rope_logical(const void *x, int64_t x_tok_stride, void *y, const 
  *   k_cache, v_cache  [pool][Hkv][block_size][d]
  *   block_table int32 [B][max_blocks]; num_tokens int32 [B] (0 gives o = 0)
  *   dt      KVS_BF16 with d = 128, or KVS_F32 with d = 64 (fp32 accumulation)
- *   ws      device scratch of kvs_paged_decode_ws_bytes(...) bytes; the call
- *           keeps a small counter area in it that it returns to zero itself;
- *           zero ws once before first use.
+ *   ws      device scratch of kvs_paged_decode_ws_bytes(...) bytes (per-split
+ *           partial results; no initialisation needed). The call runs one
+ *           split kernel and, when a sequence spans several splits, a merge
+ *           kernel.
  * A block id < 0 sets KVS_ERR_INVALID_ARG and its entries are skipped.
  */
 size_t kvs_paged_decode_ws_bytes(int32_t B, int32_t Hq, int32_t Hkv, int32_t d, int32_t block_size,
@@ -206,8 +207,7 @@ kvs_status kvs_paged_decode_attn(const void *q, const void *k_cache, const void 
  *  - Returns KVS_ERR_CAPACITY (nothing launched) when the call needs more
  *    scratch than that, i.e. kvs_paged_decode_ws_bytes(...) > the maximum.
  *  - The first call on each device looks up the array's device address
- *    (cudaGetSymbolAddress), zeroes it and synchronizes the device; make that
- *    first call before any stream capture.
+ *    (cudaGetSymbolAddress); make that first call before any stream capture.
  *  - All calls share the array: calls whose kernels overlap on the GPU
  *    (unordered streams, concurrent threads) race and give wrong results.
  *  - Allocates nothing: no cudaMalloc/cudaFree, no allocating library call.
