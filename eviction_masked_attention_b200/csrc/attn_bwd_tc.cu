@@ -258,30 +258,45 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 break;
             }
             tc_fence_after();
-            float p[64];
+            // P^T = 2^(S^T c - LSE_t log2 e) for this thread's 64 query columns, kept
+            // only as bf16 pairs (the same values the dV MMA consumes); keeping the
+            // working set small lets the scheduler overlap the independent columns
+            uint32_t pk[32];
             {
                 uint32_t r0[32], r1[32];
                 tmem_ld32(tmem + lane_off + cST + col0, r0);
                 tmem_ld32(tmem + lane_off + cST + col0 + 32, r1);
                 tmem_ld_wait();
                 const float4 *l2v = reinterpret_cast<const float4 *>(&S.l2[s][col0]);
+                const bool all_vis = rlo <= 0 && rhi >= 64;
+                if (__all_sync(0xffffffffu, all_vis)) {
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const float4 lv = l2v[i];
-                    const float ls[4] = {lv.x, lv.y, lv.z, lv.w};
+                    for (int i = 0; i < 16; ++i) {
+                        const float4 lv = l2v[i];
+                        const int rr = 4 * i;
+                        const float a0 = __uint_as_float(rr < 32 ? r0[rr] : r1[rr - 32]);
+                        const float a1 = __uint_as_float(rr < 32 ? r0[rr + 1] : r1[rr - 31]);
+                        const float a2 = __uint_as_float(rr < 32 ? r0[rr + 2] : r1[rr - 30]);
+                        const float a3 = __uint_as_float(rr < 32 ? r0[rr + 3] : r1[rr - 29]);
+                        pk[2 * i] = pack_bf16(ex2(fmaf(a0, scale_log2, -lv.x)), ex2(fmaf(a1, scale_log2, -lv.y)));
+                        pk[2 * i + 1] = pack_bf16(ex2(fmaf(a2, scale_log2, -lv.z)), ex2(fmaf(a3, scale_log2, -lv.w)));
+                    }
+                } else {
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const int rr = 4 * i + u;
-                        const uint32_t raw = rr < 32 ? r0[rr] : r1[rr - 32];
-                        const float x = __uint_as_float(raw) * scale_log2 - ls[u];
-                        p[rr] = (rr >= rlo && rr < rhi) ? ex2(x) : 0.f;
+                    for (int i = 0; i < 16; ++i) {
+                        const float4 lv = l2v[i];
+                        const float ls[4] = {lv.x, lv.y, lv.z, lv.w};
+                        float q4[4];
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const int rr = 4 * i + u;
+                            const float a = __uint_as_float(rr < 32 ? r0[rr] : r1[rr - 32]);
+                            q4[u] = (rr >= rlo && rr < rhi) ? ex2(fmaf(a, scale_log2, -ls[u])) : 0.f;
+                        }
+                        pk[2 * i] = pack_bf16(q4[0], q4[1]);
+                        pk[2 * i + 1] = pack_bf16(q4[2], q4[3]);
                     }
                 }
-            }
-            {
-                uint32_t pk[32];
-#pragma unroll
-                for (int rr = 0; rr < 64; rr += 2) pk[rr >> 1] = pack_bf16(p[rr], p[rr + 1]);
                 tmem_st32(tmem + lane_off + cST + col0, pk);
             }
             tmem_st_wait();
@@ -292,8 +307,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 break;
             }
             tc_fence_after();
+            // dS^T = P^T (dP^T - D_t), from the bf16 P^T above
             {
-                uint32_t r0[32], r1[32], pk[32];
+                uint32_t r0[32], r1[32], dk2[32];
                 tmem_ld32(tmem + lane_off + cDP + col0, r0);
                 tmem_ld32(tmem + lane_off + cDP + col0 + 32, r1);
                 tmem_ld_wait();
@@ -301,16 +317,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
                     const float4 dv4 = ddv[i];
-                    const float ds4[4] = {dv4.x, dv4.y, dv4.z, dv4.w};
-#pragma unroll
-                    for (int u = 0; u < 4; u += 2) {
-                        const int rr = 4 * i + u;
-                        const float a0 = __uint_as_float(rr < 32 ? r0[rr] : r1[rr - 32]);
-                        const float a1 = __uint_as_float(rr + 1 < 32 ? r0[rr + 1] : r1[rr + 1 - 32]);
-                        pk[rr >> 1] = pack_bf16(p[rr] * (a0 - ds4[u]), p[rr + 1] * (a1 - ds4[u + 1]));
-                    }
+                    const int rr = 4 * i;
+                    const float a0 = __uint_as_float(rr < 32 ? r0[rr] : r1[rr - 32]);
+                    const float a1 = __uint_as_float(rr < 32 ? r0[rr + 1] : r1[rr - 31]);
+                    const float a2 = __uint_as_float(rr < 32 ? r0[rr + 2] : r1[rr - 30]);
+                    const float a3 = __uint_as_float(rr < 32 ? r0[rr + 3] : r1[rr - 29]);
+                    dk2[2 * i] = pack_bf16(bf16_lo(pk[2 * i]) * (a0 - dv4.x), bf16_hi(pk[2 * i]) * (a1 - dv4.y));
+                    dk2[2 * i + 1] =
+                        pack_bf16(bf16_lo(pk[2 * i + 1]) * (a2 - dv4.z), bf16_hi(pk[2 * i + 1]) * (a3 - dv4.w));
                 }
-                tmem_st32(tmem + lane_off + cDP + col0, pk);
+                tmem_st32(tmem + lane_off + cDP + col0, dk2);
             }
             tmem_st_wait();
             tc_fence_before();
@@ -497,9 +513,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             tc_fence_after();
             // S_n complete implies stage s (K, V and the tile's mask rows) has
             // landed; it is refilled only after dQ_n, i.e. after this item's dS
+            const bool partial = S.pid[s] >= 0;  // same for the whole CTA
             uint2 bits = make_uint2(~0u, ~0u);
-            if (S.pid[s] >= 0) bits = *reinterpret_cast<const uint2 *>(&S.bits[s][row * 4 + half * 2]);
-            float p[64];
+            if (partial) bits = *reinterpret_cast<const uint2 *>(&S.bits[s][row * 4 + half * 2]);
+            // P = 2^(S c - LSE log2 e) for this thread's 64 key columns, kept as bf16
+            // pairs; dS = P (dP - D) then rounds to bf16 for the dQ MMA
+            uint32_t pp[32];
             {
                 uint32_t r0[32], r1[32];
                 tmem_ld32(tmem + lane_off + cS + col0, r0);
@@ -507,10 +526,26 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 tmem_ld_wait();
                 tc_fence_before();
                 mbar_arrive(&S.s_free);
+                if (!partial) {
 #pragma unroll
-                for (int jj = 0; jj < 32; ++jj) {
-                    p[jj] = ((bits.x >> jj) & 1u) ? ex2(__uint_as_float(r0[jj]) * scale_log2 - l2) : 0.f;
-                    p[jj + 32] = ((bits.y >> jj) & 1u) ? ex2(__uint_as_float(r1[jj]) * scale_log2 - l2) : 0.f;
+                    for (int jj = 0; jj < 32; jj += 2) {
+                        pp[jj >> 1] = pack_bf16(ex2(fmaf(__uint_as_float(r0[jj]), scale_log2, -l2)),
+                                                ex2(fmaf(__uint_as_float(r0[jj + 1]), scale_log2, -l2)));
+                        pp[16 + (jj >> 1)] = pack_bf16(ex2(fmaf(__uint_as_float(r1[jj]), scale_log2, -l2)),
+                                                       ex2(fmaf(__uint_as_float(r1[jj + 1]), scale_log2, -l2)));
+                    }
+                } else {
+#pragma unroll
+                    for (int jj = 0; jj < 32; jj += 2) {
+                        const float e0 = ex2(fmaf(__uint_as_float(r0[jj]), scale_log2, -l2));
+                        const float e1 = ex2(fmaf(__uint_as_float(r0[jj + 1]), scale_log2, -l2));
+                        const float e2 = ex2(fmaf(__uint_as_float(r1[jj]), scale_log2, -l2));
+                        const float e3 = ex2(fmaf(__uint_as_float(r1[jj + 1]), scale_log2, -l2));
+                        pp[jj >> 1] = pack_bf16(((bits.x >> jj) & 1u) ? e0 : 0.f,
+                                                ((bits.x >> (jj + 1)) & 1u) ? e1 : 0.f);
+                        pp[16 + (jj >> 1)] = pack_bf16(((bits.y >> jj) & 1u) ? e2 : 0.f,
+                                                       ((bits.y >> (jj + 1)) & 1u) ? e3 : 0.f);
+                    }
                 }
             }
             if (!warp_wait(&S.dp_full, n & 1, abort, status)) {
@@ -528,10 +563,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 mbar_arrive(&S.dp_free);
 #pragma unroll
                 for (int jj = 0; jj < 32; jj += 2) {
-                    pk[jj >> 1] = pack_bf16(p[jj] * (__uint_as_float(r0[jj]) - dd),
-                                            p[jj + 1] * (__uint_as_float(r0[jj + 1]) - dd));
-                    pk[16 + (jj >> 1)] = pack_bf16(p[jj + 32] * (__uint_as_float(r1[jj]) - dd),
-                                                   p[jj + 33] * (__uint_as_float(r1[jj + 1]) - dd));
+                    pk[jj >> 1] = pack_bf16(bf16_lo(pp[jj >> 1]) * (__uint_as_float(r0[jj]) - dd),
+                                            bf16_hi(pp[jj >> 1]) * (__uint_as_float(r0[jj + 1]) - dd));
+                    pk[16 + (jj >> 1)] = pack_bf16(bf16_lo(pp[16 + (jj >> 1)]) * (__uint_as_float(r1[jj]) - dd),
+                                                   bf16_hi(pp[16 + (jj >> 1)]) * (__uint_as_float(r1[jj + 1]) - dd));
                 }
             }
             // dQ of item n-1 must be complete: its MMA has then consumed ds_ready

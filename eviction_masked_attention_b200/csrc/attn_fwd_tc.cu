@@ -438,20 +438,36 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
                 break;
             }
             tc_fence_after();
+            const bool partial = S.pid[n & 1] >= 0;  // same for the whole CTA
             uint4 bits = make_uint4(~0u, ~0u, ~0u, ~0u);
-            if (S.pid[n & 1] >= 0) bits = *reinterpret_cast<const uint4 *>(&S.bits[n & 1][row * 4]);
+            if (partial) bits = *reinterpret_cast<const uint4 *>(&S.bits[n & 1][row * 4]);
             const uint32_t wb[4] = {bits.x, bits.y, bits.z, bits.w};
-            // pass 1: row maximum of the masked, base-2 scaled scores
-            float mt = -INFINITY;
+            // pass 1: row maximum of the (masked) raw scores; 8 independent partial
+            // maxima keep the reduction off one serial dependency chain
+            float mx8[8];
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                uint32_t r[32];
-                tmem_ld32(tmem + lane_off + cS + c * 32, r);
+            for (int u = 0; u < 8; ++u) mx8[u] = -INFINITY;
+#pragma unroll
+            for (int hc = 0; hc < 2; ++hc) {
+                uint32_t r0[32], r1[32];
+                tmem_ld32(tmem + lane_off + cS + hc * 64, r0);
+                tmem_ld32(tmem + lane_off + cS + hc * 64 + 32, r1);
                 tmem_ld_wait();
+                if (partial) {
 #pragma unroll
-                for (int j = 0; j < 32; ++j)
-                    if ((wb[c] >> j) & 1u) mt = fmaxf(mt, __uint_as_float(r[j]) * scale_log2);
+                    for (int j = 0; j < 32; ++j) {
+                        if ((wb[2 * hc] >> j) & 1u) mx8[j & 7] = fmaxf(mx8[j & 7], __uint_as_float(r0[j]));
+                        if ((wb[2 * hc + 1] >> j) & 1u) mx8[j & 7] = fmaxf(mx8[j & 7], __uint_as_float(r1[j]));
+                    }
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        mx8[j & 7] = fmaxf(mx8[j & 7], fmaxf(__uint_as_float(r0[j]), __uint_as_float(r1[j])));
+                }
             }
+            float mraw = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+            const float mt = mraw * scale_log2;  // scale_log2 > 0 keeps the order
             const float m_new = fmaxf(m_run, mt);
             float alpha = 1.f;
             bool rescale = false;
@@ -479,33 +495,42 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
                     tmem_st32(tmem + lane_off + cO + c * 32, o);
                 }
             }
-            // pass 2: P = 2^(s - m) as bf16 pairs over the first 64 columns of S
-            // (two 32-column score chunks are read before their 32 packed columns
-            // are written over the first of them)
-            const float mref = m_run == -INFINITY ? 0.f : m_run;
-            float lsum = 0.f;
+            // pass 2: P = 2^(s*c - m) as bf16 pairs over the first 64 columns of S
+            // (the two 32-column chunks of a half are read before their 32 packed
+            // columns overwrite the first of them). Half of the exponentials run on
+            // the FMA pipe (exp2_fma), half on the special-function unit.
+            const float nref = m_run == -INFINITY ? 0.f : -m_run;
+            float ls8[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) ls8[u] = 0.f;
 #pragma unroll 1
             for (int hc = 0; hc < 2; ++hc) {
-                uint32_t pk[32];
+                uint32_t r0[32], r1[32], pk[32];
+                tmem_ld32(tmem + lane_off + cS + hc * 64, r0);
+                tmem_ld32(tmem + lane_off + cS + hc * 64 + 32, r1);
+                tmem_ld_wait();
+                const uint32_t w0 = hc ? wb[2] : wb[0], w1 = hc ? wb[3] : wb[1];
 #pragma unroll
                 for (int cc = 0; cc < 2; ++cc) {
-                    const int c = 2 * hc + cc;
-                    const uint32_t w = hc ? (cc ? wb[3] : wb[2]) : (cc ? wb[1] : wb[0]);
-                    uint32_t r[32];
-                    tmem_ld32(tmem + lane_off + cS + c * 32, r);
-                    tmem_ld_wait();
+                    const uint32_t(&r)[32] = cc ? r1 : r0;
+                    const uint32_t w = cc ? w1 : w0;
 #pragma unroll
                     for (int j = 0; j < 32; j += 2) {
-                        const float s0 = __uint_as_float(r[j]) * scale_log2 - mref;
-                        const float s1 = __uint_as_float(r[j + 1]) * scale_log2 - mref;
-                        const float p0 = ((w >> j) & 1u) ? ex2(s0) : 0.f;
-                        const float p1 = ((w >> (j + 1)) & 1u) ? ex2(s1) : 0.f;
-                        lsum += p0 + p1;
+                        float x0, x1;
+                        fma2(__uint_as_float(r[j]), __uint_as_float(r[j + 1]), scale_log2, nref, x0, x1);
+                        float p0 = exp2_fma(x0);
+                        float p1 = ex2(x1);
+                        if (partial) {
+                            p0 = ((w >> j) & 1u) ? p0 : 0.f;
+                            p1 = ((w >> (j + 1)) & 1u) ? p1 : 0.f;
+                        }
+                        ls8[(j >> 1) & 7] += p0 + p1;
                         pk[cc * 16 + (j >> 1)] = pack_bf16(p0, p1);
                     }
                 }
                 tmem_st32(tmem + lane_off + cS + hc * 32, pk);
             }
+            const float lsum = ((ls8[0] + ls8[1]) + (ls8[2] + ls8[3])) + ((ls8[4] + ls8[5]) + (ls8[6] + ls8[7]));
             l_run += lsum;
             tmem_st_wait();
             tc_fence_before();

@@ -43,6 +43,44 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
+// 2^x evaluated on the FMA pipe, freeing the special-function unit (which also
+// executes conversions, so none are used): t = x + 1.5*2^23 rounds x to the
+// integer n held in the low mantissa bits of t; f = x - n lies in [-1/2, 1/2];
+// 2^f comes from a cubic fitted for minimum relative error on that interval
+// (eviction_masked_attention_b200/fit_exp2_poly.py; max relative error 1.5e-4 in
+// fp32, far below the 2^-9 of the bf16 P it feeds); n is added to the exponent
+// field by one integer multiply-add (bits(t) * 2^23 wraps to n * 2^23).
+// Arguments below -127 are clamped (result ~1e-38); valid up to x < 128.
+__device__ __forceinline__ float exp2_fma(float x) {
+    x = fmaxf(x, -127.f);
+    const float t = x + 12582912.f;
+    const float f = x - (t - 12582912.f);
+    const float p = fmaf(fmaf(fmaf(5.517166907e-02f, f, 2.426111222e-01f), f, 6.932609855e-01f), f,
+                         9.999280735e-01f);
+    return __uint_as_float(__float_as_uint(t) * 8388608u + __float_as_uint(p));
+}
+
+// Two fp32 lanes at once: (a0, a1) * (b, b) + (c, c).
+__device__ __forceinline__ void fma2(float a0, float a1, float b, float c, float &d0, float &d1) {
+    uint64_t av, bv, cv, dv;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(av) : "f"(a0), "f"(a1));
+    asm("mov.b64 %0, {%1, %1};" : "=l"(bv) : "f"(b));
+    asm("mov.b64 %0, {%1, %1};" : "=l"(cv) : "f"(c));
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(dv) : "l"(av), "l"(bv), "l"(cv));
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(d0), "=f"(d1) : "l"(dv));
+}
+
+// Two fp32 lanes at once: (a0, a1) * (b, b) + (c0, c1).
+__device__ __forceinline__ void fma2v(float a0, float a1, float b, float c0, float c1, float &d0,
+                                      float &d1) {
+    uint64_t av, bv, cv, dv;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(av) : "f"(a0), "f"(a1));
+    asm("mov.b64 %0, {%1, %1};" : "=l"(bv) : "f"(b));
+    asm("mov.b64 %0, {%1, %2};" : "=l"(cv) : "f"(c0), "f"(c1));
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(dv) : "l"(av), "l"(bv), "l"(cv));
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(d0), "=f"(d1) : "l"(dv));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&v);

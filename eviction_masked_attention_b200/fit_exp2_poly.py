@@ -1,27 +1,31 @@
-"""Derive the cubic used for 2^f, f in [0, 1), in the attention kernels.
+"""Derive the cubic used for 2^f, f in [-1/2, 1/2], in the attention kernels.
 
 The kernels evaluate part of their exponentials on the FMA pipe instead of the
-special-function unit: 2^x = 2^n * 2^f with n = floor(x), and 2^f ~ c0 + f*(c1
-+ f*(c2 + f*c3)). The coefficients minimise the maximum relative error on
-[0, 1] (a Remez exchange on the relative error, started from a least-squares
-fit at Chebyshev nodes). The result only has to beat the bf16 rounding that
-P gets before the MMA (2^-9): a cubic reaches about 9e-5.
+special-function unit: 2^x = 2^n * 2^f with n = round(x) (found by adding
+1.5 * 2^23, which needs no conversion instruction), and 2^f ~ c0 + f*(c1 +
+f*(c2 + f*c3)). The coefficients minimise the maximum relative error on
+[-1/2, 1/2] (a Remez exchange on the relative error, started from a least-
+squares fit at Chebyshev nodes). The result only has to beat the bf16 rounding
+that P gets before the MMA (2^-9): a cubic reaches about 9e-5.
 
 Run: python -m eviction_masked_attention_b200.fit_exp2_poly
 """
 import numpy as np
 
 
+LO, HI = -0.5, 0.5
+
+
 def fit(deg: int = 3, iters: int = 30):
     # initial least-squares fit of the relative error at Chebyshev nodes
     n = 64
-    x = 0.5 - 0.5 * np.cos(np.pi * (np.arange(n) + 0.5) / n)
+    x = 0.5 * (LO + HI) - 0.5 * (HI - LO) * np.cos(np.pi * (np.arange(n) + 0.5) / n)
     y = np.exp2(x)
     A = np.vander(x, deg + 1, increasing=True) / y[:, None]
     c = np.linalg.lstsq(A, np.ones(n), rcond=None)[0]
     # Remez exchange on e(x) = p(x)/2^x - 1 with deg + 2 reference points
-    ref = 0.5 - 0.5 * np.cos(np.pi * np.arange(deg + 2) / (deg + 1))
-    grid = np.linspace(0.0, 1.0, 20001)
+    ref = 0.5 * (LO + HI) - 0.5 * (HI - LO) * np.cos(np.pi * np.arange(deg + 2) / (deg + 1))
+    grid = np.linspace(LO, HI, 20001)
     for _ in range(iters):
         yr = np.exp2(ref)
         M = np.zeros((deg + 2, deg + 2))
@@ -40,16 +44,25 @@ def fit(deg: int = 3, iters: int = 30):
     return c, float(np.abs(err).max())
 
 
-def fp32_error(c):
-    """Max relative error of the kernel's fp32 evaluation over x in [-126, 0]."""
-    x = np.linspace(-126.0, 0.0, 2_000_001).astype(np.float32)
+MAGIC = np.float32(12582912.0)  # 1.5 * 2^23: x + MAGIC rounds x to an integer
+
+
+def eval_fp32(c, x):
+    """The kernels' fp32 evaluation: t = x + MAGIC (round to nearest), f = x - (t - MAGIC),
+    p = cubic(f), result bits = bits(p) + bits(t) * 2^23 (mod 2^32)."""
     cf = c.astype(np.float32)
-    nfl = np.floor(x)
-    f = (x - nfl).astype(np.float32)
-    p = ((cf[3] * f + cf[2]) * f + cf[1]) * f + cf[0]
-    p = p.astype(np.float32)
-    bits = p.view(np.int32) + (nfl.astype(np.int32) << 23)
-    got = bits.view(np.float32).astype(np.float64)
+    x = np.maximum(np.asarray(x, dtype=np.float32), np.float32(-127.0))
+    t = (x + MAGIC).astype(np.float32)
+    f = (x - (t - MAGIC)).astype(np.float32)
+    p = (((cf[3] * f + cf[2]) * f + cf[1]) * f + cf[0]).astype(np.float32)
+    bits = (p.view(np.uint32).astype(np.uint64) + (t.view(np.uint32).astype(np.uint64) << 23)) & 0xFFFFFFFF
+    return bits.astype(np.uint32).view(np.float32)
+
+
+def fp32_error(c):
+    """Max relative error of the kernel's fp32 evaluation over x in [-126, 8]."""
+    x = np.linspace(-126.0, 8.0, 2_000_001).astype(np.float32)
+    got = eval_fp32(c, x).astype(np.float64)
     want = np.exp2(x.astype(np.float64))
     return float(np.max(np.abs(got / want - 1.0)))
 

@@ -1,0 +1,42 @@
+"""The cubic 2^x the attention kernels evaluate on the FMA pipe: its constants
+in csrc/common.cuh are the ones eviction_masked_attention_b200/fit_exp2_poly.py
+derives, and its fp32 evaluation stays within 2e-4 relative error of 2^x over
+the arguments the kernels use (scores minus the running maximum, which the lazy
+rescale lets reach +8)."""
+import os
+import re
+
+import numpy as np
+
+from eviction_masked_attention_b200 import fit_exp2_poly
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _kernel_coeffs():
+    src = open(os.path.join(ROOT, "eviction_masked_attention_b200", "csrc", "common.cuh")).read()
+    body = src[src.index("float exp2_fma("):]
+    body = body[body.index("const float p"): body.index("return")]
+    vals = [float(v) for v in re.findall(r"([0-9]\.[0-9]+e[+-][0-9]+)f", body)]
+    c3, c2, c1, c0 = vals[:4]
+    return np.array([c0, c1, c2, c3])
+
+
+def _eval_fp32(c, x):
+    return fit_exp2_poly.eval_fp32(c, x)
+
+
+def test_constants_match_fit():
+    c, err = fit_exp2_poly.fit()
+    np.testing.assert_allclose(_kernel_coeffs(), c, rtol=1e-8)
+    assert err < 1e-4
+
+
+def test_relative_error_over_kernel_range():
+    c = _kernel_coeffs()
+    x = np.concatenate([np.linspace(-126.0, 8.0, 1_000_001), -np.arange(0, 127), [0.5, -0.5, 7.999]])
+    got = _eval_fp32(c, x).astype(np.float64)
+    want = np.exp2(x.astype(np.float32).astype(np.float64))
+    assert np.max(np.abs(got / want - 1.0)) < 2e-4
+    # exact powers of two stay within the same bound
+    assert abs(_eval_fp32(c, np.array([0.0]))[0] - 1.0) < 2e-4
