@@ -24,7 +24,7 @@
 
 namespace kvs {
 
-bool make_tmap_bnhd(CUtensorMap *map, const void *base, int B, int N, int H);
+bool make_tmap_bnhd(CUtensorMap *map, const void *base, int B, int N, int H, int box_rows);
 
 constexpr uint32_t kTile = 128 * 128 * 2;
 
@@ -93,18 +93,29 @@ __device__ __forceinline__ void store_row64(__nv_bfloat16 *dst, const uint32_t (
 __device__ __forceinline__ uint32_t packed_col(int kk) { return (kk < 4) ? kk * 8 : 64 + (kk - 4) * 8; }
 
 // ---------------------------------------------------------------------- dK / dV
+//
+// An item is (64-row query half-tile, query head of the group); a CTA walks the
+// items of its key tile: for each listed query tile, each head, both halves.
+// TMEM: S^T in two 64-column buffers [0,64) [64,128), dP^T in two more
+// [128,192) [192,256), dV [256,384), dK [384,512). Two groups of four
+// elementwise warps take the items in turn (group = item parity = buffer), so
+// while one group forms P^T and dS^T of item n the tensor core computes S^T and
+// dP^T of item n+1 and the accumulations of item n-1.
 
 constexpr int kBwdThreads = 320;  // warp 0 TMA, warp 1 MMA, warps 2..9 elementwise
+constexpr int kDkvStages = 4;
+constexpr uint32_t kHalfTile = 64 * 128 * 2;  // 64 rows x 128 dims, bf16
 
 struct DkvSmem {
     uint8_t k[kTile];
     uint8_t v[kTile];
-    uint8_t q[2][kTile];
-    uint8_t dout[2][kTile];
-    float l2[2][128];
-    float dd[2][128];
-    int32_t q0[2], full_tile[2];  // query tile origin and FULL flag of the item in each stage
-    uint64_t kv_full, full[2], empty[2], st_full, dp_full, p_ready, ds_ready, acc_done, fin;
+    uint8_t q[kDkvStages][kHalfTile];
+    uint8_t dout[kDkvStages][kHalfTile];
+    float l2[kDkvStages][64];
+    float dd[kDkvStages][64];
+    int32_t q0[kDkvStages], full_tile[kDkvStages];  // half-tile origin, FULL flag of its tile
+    uint64_t kv_full, full[kDkvStages], empty[kDkvStages], st_full[2], dp_full[2], p_ready[2],
+        ds_ready[2], acc_done, fin;
     uint32_t tmem_base;
     int abort;
 };
@@ -127,19 +138,21 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int kvh = rem % Hkv, b = rem / Hkv;
     const int k0 = kj * 128;
     const int32_t c0 = m.col_ptr[b * T + kj], ncol = m.col_ptr[b * T + kj + 1] - c0;
-    const int nw = ncol * G;
+    const int nw = ncol * G * 2;
     if (grid_timed_out(status)) return;
 
     if (threadIdx.x == 0) {
         mbar_init(&S.kv_full, 1);
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < kDkvStages; ++i) {
             mbar_init(&S.full[i], 1);
             mbar_init(&S.empty[i], 1);
         }
-        mbar_init(&S.st_full, 1);
-        mbar_init(&S.dp_full, 1);
-        mbar_init(&S.p_ready, 256);
-        mbar_init(&S.ds_ready, 256);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&S.st_full[i], 1);
+            mbar_init(&S.dp_full[i], 1);
+            mbar_init(&S.p_ready[i], 128);
+            mbar_init(&S.ds_ready[i], 128);
+        }
         mbar_init(&S.acc_done, 1);
         mbar_init(&S.fin, 1);
         S.abort = 0;
@@ -164,110 +177,126 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             tma_load_4d(S.v, &tmV, &S.kv_full, 0, kvh, k0, b);
             tma_load_4d(S.v + kTile / 2, &tmV, &S.kv_full, 64, kvh, k0, b);
             for (int n = 0; n < nw; ++n) {
-                const int s = n & 1;
-                if (n >= 2 && !mbar_wait(&S.empty[s], ((n >> 1) - 1) & 1, abort, status)) break;
-                const int e = n / G, g = n % G, h = kvh * G + g;
-                const int q0 = m.col_row[c0 + e] * 128;
+                const int s = n % kDkvStages;
+                if (n >= kDkvStages &&
+                    !mbar_wait(&S.empty[s], ((n / kDkvStages) - 1) & 1, abort, status))
+                    break;
+                const int e = n / (2 * G), r = n % (2 * G), h = kvh * G + (r >> 1);
+                const int q0 = m.col_row[c0 + e] * 128 + (r & 1) * 64;
                 S.q0[s] = q0;
                 S.full_tile[s] = m.col_pidx[c0 + e] < 0;
-                mbar_expect_tx(&S.full[s], 2 * kTile + 1024);
+                mbar_expect_tx(&S.full[s], 2 * kHalfTile + 512);
                 tma_load_4d(S.q[s], &tmQ, &S.full[s], 0, h, q0, b);
-                tma_load_4d(S.q[s] + kTile / 2, &tmQ, &S.full[s], 64, h, q0, b);
+                tma_load_4d(S.q[s] + kHalfTile / 2, &tmQ, &S.full[s], 64, h, q0, b);
                 tma_load_4d(S.dout[s], &tmO, &S.full[s], 0, h, q0, b);
-                tma_load_4d(S.dout[s] + kTile / 2, &tmO, &S.full[s], 64, h, q0, b);
+                tma_load_4d(S.dout[s] + kHalfTile / 2, &tmO, &S.full[s], 64, h, q0, b);
                 const int64_t ro = ((int64_t)b * Hq + h) * Tpad + q0;
-                bulk_load(S.l2[s], L2 + ro, 512, &S.full[s]);
-                bulk_load(S.dd[s], Drow + ro, 512, &S.full[s]);
+                bulk_load(S.l2[s], L2 + ro, 256, &S.full[s]);
+                bulk_load(S.dd[s], Drow + ro, 256, &S.full[s]);
             }
         }
     } else if (warp == 1) {
         if (lane == 0 && nw > 0) {
-            const uint32_t idKM = idesc_bf16(128, 128, false, false);  // both K-major
-            const uint32_t idMN = idesc_bf16(128, 128, false, true);   // B MN-major
-            const uint32_t ka = smem_u32(S.k), va = smem_u32(S.v);
-            bool ok = mbar_wait(&S.kv_full, 0, abort, status);
+            const uint32_t idT = idesc_bf16(128, 64, false, false);   // S^T, dP^T: both K-major
+            const uint32_t idMN = idesc_bf16(128, 128, false, true);  // dV, dK: B MN-major
+            const uint64_t kd = sw128_desc(smem_u32(S.k), 16, 1024);
+            const uint64_t vd = sw128_desc(smem_u32(S.v), 16, 1024);
+            // stage 0 of Q and dO as K-major (B of S^T, dP^T) and MN-major (B of dK, dV)
+            const uint64_t qk0 = sw128_desc(smem_u32(S.q[0]), 16, 1024);
+            const uint64_t ok0 = sw128_desc(smem_u32(S.dout[0]), 16, 1024);
+            const uint64_t qm0 = sw128_desc(smem_u32(S.q[0]), kHalfTile / 2, 1024);
+            const uint64_t om0 = sw128_desc(smem_u32(S.dout[0]), kHalfTile / 2, 1024);
+            // S^T = K Q^T and dP^T = V dO^T of item n into buffer n & 1
+            auto issue_t = [&](int n) -> bool {
+                const int s = n % kDkvStages;
+                const uint32_t buf = (uint32_t)(n & 1) * 64;
+                if (!mbar_wait(&S.full[s], (n / kDkvStages) & 1, abort, status)) return false;
+                tc_fence_after();
+                const uint64_t qd = desc_add(qk0, s * kHalfTile), od = desc_add(ok0, s * kHalfTile);
+                const uint32_t dst = tmem + cST + buf, ddp = tmem + cDP + buf;
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t offa = (kk >> 2) * (kTile / 2) + (kk & 3) * 32;
+                    const uint32_t offb = (kk >> 2) * (kHalfTile / 2) + (kk & 3) * 32;
+                    mma_ss(dst, desc_add(kd, offa), desc_add(qd, offb), idT, kk > 0);
+                }
+                mma_commit(&S.st_full[n & 1]);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t offa = (kk >> 2) * (kTile / 2) + (kk & 3) * 32;
+                    const uint32_t offb = (kk >> 2) * (kHalfTile / 2) + (kk & 3) * 32;
+                    mma_ss(ddp, desc_add(vd, offa), desc_add(od, offb), idT, kk > 0);
+                }
+                mma_commit(&S.dp_full[n & 1]);
+                return true;
+            };
+            bool ok = mbar_wait(&S.kv_full, 0, abort, status) && issue_t(0) && (nw < 2 || issue_t(1));
             for (int n = 0; ok && n < nw; ++n) {
-                const int s = n & 1;
-                if (!mbar_wait(&S.full[s], (n >> 1) & 1, abort, status)) break;
-                tc_fence_after();
-                const uint32_t qa = smem_u32(S.q[s]), oa = smem_u32(S.dout[s]);
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t off = (kk >> 2) * (kTile / 2) + (kk & 3) * 32;
-                    mma_ss(tmem + cST, sw128_desc(ka + off, 16, 1024), sw128_desc(qa + off, 16, 1024),
-                           idKM, kk > 0);
-                }
-                mma_commit(&S.st_full);
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t off = (kk >> 2) * (kTile / 2) + (kk & 3) * 32;
-                    mma_ss(tmem + cDP, sw128_desc(va + off, 16, 1024), sw128_desc(oa + off, 16, 1024),
-                           idKM, kk > 0);
-                }
-                mma_commit(&S.dp_full);
-                if (!mbar_wait(&S.p_ready, n & 1, abort, status)) break;
+                const int s = n % kDkvStages;
+                const uint32_t buf = (uint32_t)(n & 1) * 64;
+                const uint64_t qm = desc_add(qm0, s * kHalfTile), om = desc_add(om0, s * kHalfTile);
+                const uint32_t pa = tmem + cST + buf, sa = tmem + cDP + buf, acc = n > 0 ? 1u : 0u;
+                if (!mbar_wait(&S.p_ready[n & 1], (n >> 1) & 1, abort, status)) break;
                 tc_fence_after();
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_ts(tmem + cDV, tmem + cST + packed_col(kk),
-                           sw128_desc(oa + kk * 2048, kTile / 2, 1024), idMN, (n > 0 || kk > 0) ? 1u : 0u);
-                if (!mbar_wait(&S.ds_ready, n & 1, abort, status)) break;
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_ts(tmem + cDV, pa + kk * 8, desc_add(om, kk * 2048), idMN, kk > 0 ? 1u : acc);
+                if (!mbar_wait(&S.ds_ready[n & 1], (n >> 1) & 1, abort, status)) break;
                 tc_fence_after();
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_ts(tmem + cDK, tmem + cDP + packed_col(kk),
-                           sw128_desc(qa + kk * 2048, kTile / 2, 1024), idMN, (n > 0 || kk > 0) ? 1u : 0u);
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_ts(tmem + cDK, sa + kk * 8, desc_add(qm, kk * 2048), idMN, kk > 0 ? 1u : acc);
                 mma_commit(&S.empty[s]);
+                // the products of item n+2 reuse this buffer: the MMAs above, which
+                // read P^T and dS^T from it, were issued first and run in order
+                if (n + 2 < nw && !issue_t(n + 2)) break;
             }
             mma_commit(&S.acc_done);
             mma_commit(&S.fin);
             wait_done(&S.fin, 0);
         }
     } else {
-        // thread = key row c (TMEM lane), half = which 64 query columns it handles
-        const int quad = warp & 3, half = (warp - 2) >> 2;
+        // thread = key row c (TMEM lane); group = item parity = TMEM buffer
+        const int quad = warp & 3, group = (warp - 2) >> 2;
         const int c = quad * 32 + lane;
         const int j = k0 + c;
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-        const uint32_t col0 = half * 64;
+        const uint32_t colS = cST + group * 64, colP = cDP + group * 64;
         const int32_t kap = j < N ? m.kappa[(int64_t)b * N + j] : 0;
         bool ok = true;
-        for (int n = 0; n < nw; ++n) {
-            const int s = n & 1;
-            if (!warp_wait(&S.full[s], (n >> 1) & 1, abort, status)) {
+        for (int n = group; n < nw; n += 2) {
+            const int s = n % kDkvStages;
+            const uint32_t ph = (n >> 1) & 1;
+            if (!warp_wait(&S.full[s], (n / kDkvStages) & 1, abort, status)) {
                 ok = false;
                 break;
             }
             const int q0 = S.q0[s];
-            const bool full = S.full_tile[s] != 0;
-            // visible query rows of this key inside the tile: [rlo, rhi) (j <= t < kappa_j)
-            int rlo = 0, rhi = 128;
-            if (!full) {
+            // visible query rows of this key inside the half-tile: [rlo, rhi) (j <= t < kappa_j)
+            int rlo = 0, rhi = 64;
+            if (!S.full_tile[s]) {
                 if (j >= N) {
                     rlo = rhi = 0;
                 } else {
                     const int64_t lo = (int64_t)j - q0, hi = (int64_t)(kap < N ? kap : N) - q0;
-                    rlo = (int)(lo < 0 ? 0 : (lo > 128 ? 128 : lo));
-                    rhi = (int)(hi < 0 ? 0 : (hi > 128 ? 128 : hi));
+                    rlo = (int)(lo < 0 ? 0 : (lo > 64 ? 64 : lo));
+                    rhi = (int)(hi < 0 ? 0 : (hi > 64 ? 64 : hi));
                 }
             }
-            rlo -= col0;
-            rhi -= col0;
-            if (!warp_wait(&S.st_full, n & 1, abort, status)) {
+            if (!warp_wait(&S.st_full[group], ph, abort, status)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            // P^T = 2^(S^T c - LSE_t log2 e) for this thread's 64 query columns, kept
-            // only as bf16 pairs (the same values the dV MMA consumes); keeping the
-            // working set small lets the scheduler overlap the independent columns
+            // P^T = 2^(S^T c - LSE_t log2 e), kept only as bf16 pairs (the values the
+            // dV MMA consumes)
             uint32_t pk[32];
             {
                 uint32_t r0[32], r1[32];
-                tmem_ld32(tmem + lane_off + cST + col0, r0);
-                tmem_ld32(tmem + lane_off + cST + col0 + 32, r1);
+                tmem_ld32(tmem + lane_off + colS, r0);
+                tmem_ld32(tmem + lane_off + colS + 32, r1);
                 tmem_ld_wait();
-                const float4 *l2v = reinterpret_cast<const float4 *>(&S.l2[s][col0]);
+                const float4 *l2v = reinterpret_cast<const float4 *>(S.l2[s]);
                 const bool all_vis = rlo <= 0 && rhi >= 64;
                 if (__all_sync(0xffffffffu, all_vis)) {
 #pragma unroll
@@ -297,12 +326,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                         pk[2 * i + 1] = pack_bf16(q4[2], q4[3]);
                     }
                 }
-                tmem_st32(tmem + lane_off + cST + col0, pk);
+                tmem_st32(tmem + lane_off + colS, pk);
             }
             tmem_st_wait();
             tc_fence_before();
-            mbar_arrive(&S.p_ready);
-            if (!warp_wait(&S.dp_full, n & 1, abort, status)) {
+            mbar_arrive(&S.p_ready[group]);
+            if (!warp_wait(&S.dp_full[group], ph, abort, status)) {
                 ok = false;
                 break;
             }
@@ -310,10 +339,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             // dS^T = P^T (dP^T - D_t), from the bf16 P^T above
             {
                 uint32_t r0[32], r1[32], dk2[32];
-                tmem_ld32(tmem + lane_off + cDP + col0, r0);
-                tmem_ld32(tmem + lane_off + cDP + col0 + 32, r1);
+                tmem_ld32(tmem + lane_off + colP, r0);
+                tmem_ld32(tmem + lane_off + colP + 32, r1);
                 tmem_ld_wait();
-                const float4 *ddv = reinterpret_cast<const float4 *>(&S.dd[s][col0]);
+                const float4 *ddv = reinterpret_cast<const float4 *>(S.dd[s]);
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
                     const float4 dv4 = ddv[i];
@@ -326,12 +355,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     dk2[2 * i + 1] =
                         pack_bf16(bf16_lo(pk[2 * i + 1]) * (a2 - dv4.z), bf16_hi(pk[2 * i + 1]) * (a3 - dv4.w));
                 }
-                tmem_st32(tmem + lane_off + cDP + col0, dk2);
+                tmem_st32(tmem + lane_off + colP, dk2);
             }
             tmem_st_wait();
             tc_fence_before();
-            mbar_arrive(&S.ds_ready);
+            mbar_arrive(&S.ds_ready[group]);
         }
+        // each group writes 64 of the 128 dimensions of dV and dK
+        const uint32_t col0 = group * 64;
         if (ok && nw > 0 && warp_wait(&S.acc_done, 0, abort, status)) {
             tc_fence_after();
             const int64_t ro = (((int64_t)b * N + j) * Hkv + kvh) * 128 + col0;
@@ -451,18 +482,24 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (lane == 0 && nt > 0) {
             const uint32_t idKM = idesc_bf16(128, 128, false, false);
             const uint32_t idMN = idesc_bf16(128, 128, false, true);
-            const uint32_t qa = smem_u32(S.q), oa = smem_u32(S.dout);
+            const uint64_t qd = sw128_desc(smem_u32(S.q), 16, 1024);
+            const uint64_t od = sw128_desc(smem_u32(S.dout), 16, 1024);
+            const uint64_t kd0 = sw128_desc(smem_u32(S.k[0]), 16, 1024);
+            const uint64_t kd1 = sw128_desc(smem_u32(S.k[1]), 16, 1024);
+            const uint64_t vd0 = sw128_desc(smem_u32(S.v[0]), 16, 1024);
+            const uint64_t vd1 = sw128_desc(smem_u32(S.v[1]), 16, 1024);
+            const uint64_t km0 = sw128_desc(smem_u32(S.k[0]), kTile / 2, 1024);
+            const uint64_t km1 = sw128_desc(smem_u32(S.k[1]), kTile / 2, 1024);
             auto issue_s_dp = [&](int n) -> bool {
                 const int s = n & 1;
                 if (!mbar_wait(&S.full[s], (n >> 1) & 1, abort, status)) return false;
-                const uint32_t ka = smem_u32(S.k[s]), va = smem_u32(S.v[s]);
+                const uint64_t kd = s ? kd1 : kd0, vd = s ? vd1 : vd0;
                 if (n > 0 && !mbar_wait(&S.s_free, (n - 1) & 1, abort, status)) return false;
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint32_t off = (kk >> 2) * (kTile / 2) + (kk & 3) * 32;
-                    mma_ss(tmem + cS, sw128_desc(qa + off, 16, 1024), sw128_desc(ka + off, 16, 1024),
-                           idKM, kk > 0);
+                    mma_ss(tmem + cS, desc_add(qd, off), desc_add(kd, off), idKM, kk > 0);
                 }
                 mma_commit(&S.s_full);
                 if (n > 0 && !mbar_wait(&S.dp_free, (n - 1) & 1, abort, status)) return false;
@@ -470,8 +507,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint32_t off = (kk >> 2) * (kTile / 2) + (kk & 3) * 32;
-                    mma_ss(tmem + cDP, sw128_desc(oa + off, 16, 1024), sw128_desc(va + off, 16, 1024),
-                           idKM, kk > 0);
+                    mma_ss(tmem + cDP, desc_add(od, off), desc_add(vd, off), idKM, kk > 0);
                 }
                 mma_commit(&S.dp_full);
                 return true;
@@ -482,11 +518,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 if (n + 1 < nt && !issue_s_dp(n + 1)) break;
                 if (!mbar_wait(&S.ds_ready, n & 1, abort, status)) break;
                 tc_fence_after();
-                const uint32_t ka = smem_u32(S.k[s]);
+                const uint64_t km = s ? km1 : km0;
+                const uint32_t sa = tmem + cDS + s * 64, acc = n > 0 ? 1u : 0u;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    mma_ts(tmem + cDQ, tmem + cDS + s * 64 + kk * 8,
-                           sw128_desc(ka + kk * 2048, kTile / 2, 1024), idMN, (n > 0 || kk > 0) ? 1u : 0u);
+                    mma_ts(tmem + cDQ, sa + kk * 8, desc_add(km, kk * 2048), idMN, kk > 0 ? 1u : acc);
                 mma_commit(&S.empty[s]);
                 mma_commit(&S.dq_done);
             }
@@ -606,9 +642,10 @@ cudaError_t launch_bwd_tc(const void *q, const void *k, const void *v, const voi
                           const void *o_lo, const void *dO, const float *lse, const kvs_tile_mask &m, int32_t Hq,
                           int32_t Hkv, float scale, void *dq, void *dk, void *dv, void *ws,
                           int32_t stages, int32_t *status, cudaStream_t s, bool *map_ok) {
-    CUtensorMap tq, tk, tv, to;
-    *map_ok = make_tmap_bnhd(&tq, q, m.B, m.N, Hq) && make_tmap_bnhd(&tk, k, m.B, m.N, Hkv) &&
-              make_tmap_bnhd(&tv, v, m.B, m.N, Hkv) && make_tmap_bnhd(&to, dO, m.B, m.N, Hq);
+    CUtensorMap tq, tk, tv, to, tq64, to64;
+    *map_ok = make_tmap_bnhd(&tq, q, m.B, m.N, Hq, 128) && make_tmap_bnhd(&tk, k, m.B, m.N, Hkv, 128) &&
+              make_tmap_bnhd(&tv, v, m.B, m.N, Hkv, 128) && make_tmap_bnhd(&to, dO, m.B, m.N, Hq, 128) &&
+              make_tmap_bnhd(&tq64, q, m.B, m.N, Hq, 64) && make_tmap_bnhd(&to64, dO, m.B, m.N, Hq, 64);
     if (!*map_ok) return cudaSuccess;
     const int32_t Tpad = m.T * 128;
     float *Drow = (float *)ws;
@@ -626,7 +663,7 @@ cudaError_t launch_bwd_tc(const void *q, const void *k, const void *v, const voi
                                  (int)smem);
         if (e != cudaSuccess) return e;
         k_attn_dkdv_tc<<<(unsigned)((int64_t)m.B * Hkv * m.T), kBwdThreads, smem, s>>>(
-            tq, tk, tv, to, m, Hq, Hkv, scale, sl2, Drow, L2, (__nv_bfloat16 *)dk,
+            tq64, tk, tv, to64, m, Hq, Hkv, scale, sl2, Drow, L2, (__nv_bfloat16 *)dk,
             (__nv_bfloat16 *)dv, status);
     }
     if (stages & KVS_BWD_DQ) {

@@ -111,18 +111,22 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         if (lane == 0 && nt > 0) {
             const uint32_t idS = idesc_bf16(128, 128, false, false);
             const uint32_t idPV = idesc_bf16(128, 128, false, true);
-            const uint32_t qa = smem_u32(S.q);
+            const uint64_t qd = sw128_desc(smem_u32(S.q), 16, 1024);
+            const uint64_t kd0 = sw128_desc(smem_u32(S.k[0]), 16, 1024);
+            const uint64_t kd1 = sw128_desc(smem_u32(S.k[1]), 16, 1024);
+            const uint64_t vd0 = sw128_desc(smem_u32(S.v[0]), kTileBytes / 2, 1024);
+            const uint64_t vd1 = sw128_desc(smem_u32(S.v[1]), kTileBytes / 2, 1024);
             bool ok = mbar_wait(&S.bar_q, 0, abort, status);
             auto issue_s = [&](int n) -> bool {
                 const int s = n & 1;
                 if (!mbar_wait(&S.kfull[s], (n >> 1) & 1, abort, status)) return false;
                 tc_fence_after();
-                const uint32_t ka = smem_u32(S.k[s]);
+                const uint64_t kd = s ? kd1 : kd0;
+                const uint32_t d = tmem + s * 128;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint32_t off = (kk >> 2) * (kTileBytes / 2) + (kk & 3) * 32;
-                    mma_ss(tmem + s * 128, sw128_desc(qa + off, 16, 1024),
-                           sw128_desc(ka + off, 16, 1024), idS, kk > 0);
+                    mma_ss(d, desc_add(qd, off), desc_add(kd, off), idS, kk > 0);
                 }
                 mma_commit(&S.kempty[s]);
                 mma_commit(&S.sfull[s]);
@@ -135,12 +139,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 if (!mbar_wait(&S.pfull[s], (n >> 1) & 1, abort, status)) break;
                 if (!mbar_wait(&S.vfull[s], (n >> 1) & 1, abort, status)) break;
                 tc_fence_after();
-                const uint32_t va = smem_u32(S.v[s]);
+                const uint64_t vd = s ? vd1 : vd0;
+                const uint32_t pa = tmem + s * 128, acc = n > 0 ? 1u : 0u;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    mma_ts(tmem + 256, tmem + s * 128 + kk * 8,
-                           sw128_desc(va + kk * 2048, kTileBytes / 2, 1024), idPV,
-                           (n > 0 || kk > 0) ? 1u : 0u);
+                    mma_ts(tmem + 256, pa + kk * 8, desc_add(vd, kk * 2048), idPV, kk > 0 ? 1u : acc);
                 mma_commit(&S.vempty[s]);
                 mma_commit(&S.odone);
             }
@@ -367,23 +370,28 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
         if (lane == 0 && nt > 0) {
             const uint32_t idS = idesc_bf16(128, 128, false, false);
             const uint32_t idPV = idesc_bf16(128, 128, false, true);
+            const uint64_t qd0 = sw128_desc(smem_u32(S.q[0]), 16, 1024);
+            const uint64_t qd1 = sw128_desc(smem_u32(S.q[1]), 16, 1024);
+            const uint64_t kd0 = sw128_desc(smem_u32(S.k[0]), 16, 1024);
+            const uint64_t kd1 = sw128_desc(smem_u32(S.k[1]), 16, 1024);
+            const uint64_t vd0 = sw128_desc(smem_u32(S.v[0]), kTileBytes / 2, 1024);
+            const uint64_t vd1 = sw128_desc(smem_u32(S.v[1]), kTileBytes / 2, 1024);
             auto issue_s = [&](int x, int n) {
-                const uint32_t qa = smem_u32(S.q[x]), ka = smem_u32(S.k[n & 1]);
+                const uint64_t qd = x ? qd1 : qd0, kd = (n & 1) ? kd1 : kd0;
+                const uint32_t d = tmem + x * 128;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint32_t off = (kk >> 2) * (kTileBytes / 2) + (kk & 3) * 32;
-                    mma_ss(tmem + x * 128, sw128_desc(qa + off, 16, 1024),
-                           sw128_desc(ka + off, 16, 1024), idS, kk > 0);
+                    mma_ss(d, desc_add(qd, off), desc_add(kd, off), idS, kk > 0);
                 }
                 mma_commit(&S.sfull[x]);
             };
             auto issue_pv = [&](int x, int n) {
-                const uint32_t va = smem_u32(S.v[n & 1]);
+                const uint64_t vd = (n & 1) ? vd1 : vd0;
+                const uint32_t d = tmem + 256 + x * 128, pa = tmem + x * 128, acc = n > 0 ? 1u : 0u;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    mma_ts(tmem + 256 + x * 128, tmem + x * 128 + kk * 8,
-                           sw128_desc(va + kk * 2048, kTileBytes / 2, 1024), idPV,
-                           (n > 0 || kk > 0) ? 1u : 0u);
+                    mma_ts(d, pa + kk * 8, desc_add(vd, kk * 2048), idPV, kk > 0 ? 1u : acc);
                 mma_commit(&S.odone[x]);
             };
             bool ok = mbar_wait(&S.bar_q, 0, abort, status) &&
@@ -597,12 +605,13 @@ EncodeTiledFn get_encode_fn() {
 }
 
 // [B][N][H][128] bf16 viewed as 4-D (d, H, N, B); box = 64 x 1 x 128 x 1, 128-B swizzle.
-bool make_tmap_bnhd(CUtensorMap *map, const void *base, int B, int N, int H) {
+// [B, N, H, 128] bf16, boxes of 64 dims x box_rows tokens of one head, 128-byte swizzle.
+bool make_tmap_bnhd(CUtensorMap *map, const void *base, int B, int N, int H, int box_rows) {
     EncodeTiledFn enc = get_encode_fn();
     if (!enc) return false;
     cuuint64_t dims[4] = {128, (cuuint64_t)H, (cuuint64_t)N, (cuuint64_t)B};
     cuuint64_t strides[3] = {128 * 2, (cuuint64_t)H * 256, (cuuint64_t)N * H * 256};
-    cuuint32_t box[4] = {64, 1, 128, 1};
+    cuuint32_t box[4] = {64, 1, (cuuint32_t)box_rows, 1};
     cuuint32_t estr[4] = {1, 1, 1, 1};
     CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims,
                      strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -614,8 +623,8 @@ cudaError_t launch_fwd_tc(const void *q, const void *k, const void *v, const kvs
                           int32_t Hq, int32_t Hkv, float scale, void *o, void *o_lo, float *lse,
                           int32_t *status, cudaStream_t s, bool *map_ok) {
     CUtensorMap tq, tk, tv;
-    *map_ok = make_tmap_bnhd(&tq, q, m.B, m.N, Hq) && make_tmap_bnhd(&tk, k, m.B, m.N, Hkv) &&
-              make_tmap_bnhd(&tv, v, m.B, m.N, Hkv);
+    *map_ok = make_tmap_bnhd(&tq, q, m.B, m.N, Hq, 128) && make_tmap_bnhd(&tk, k, m.B, m.N, Hkv, 128) &&
+              make_tmap_bnhd(&tv, v, m.B, m.N, Hkv, 128);
     if (!*map_ok) return cudaSuccess;
     const int G = Hq / Hkv;
     const float sl2 = scale * 1.4426950408889634f;

@@ -289,6 +289,13 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo, uin
     return d;
 }
 
+// Advance a shared-memory matrix descriptor by a byte offset. The start address
+// field counts 16-byte units and every shared address fits in it, so the sum
+// does not carry into the neighbouring fields. Issuing each MMA from a base
+// descriptor plus a compile-time offset keeps the issuing thread's work per
+// tcgen05.mma to a single add.
+__device__ __forceinline__ uint64_t desc_add(uint64_t d, uint32_t bytes) { return d + (bytes >> 4); }
+
 // Instruction descriptor: kind::f16, bf16 A and B, fp32 D, dense, M x N.
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn_major, bool b_mn_major) {
     return (1u << 4)                       // D format fp32
