@@ -35,10 +35,6 @@ __device__ __forceinline__ bool wait_done(uint64_t *bar, uint32_t parity) {
     return true;
 }
 
-__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
-                                          int32_t *status) {
-    return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, status));
-}
 
 // D[b][h][t] = <dO, O>, L2[b][h][t] = lse * log2(e); rows t >= N get 0. Tpad = T*128.
 // O is o_hi (+ o_lo when the forward kept the rounding residual of its output).
@@ -196,7 +192,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             }
         }
     } else if (warp == 1) {
-        if (lane == 0 && nw > 0) {
+        if (nw > 0) {
+            const bool leader = elect_one();
             const uint32_t idT = idesc_bf16(128, 64, false, false);   // S^T, dP^T: both K-major
             const uint32_t idMN = idesc_bf16(128, 128, false, true);  // dV, dK: B MN-major
             const uint64_t kd = sw128_desc(smem_u32(S.k), 16, 1024);
@@ -206,53 +203,66 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             const uint64_t ok0 = sw128_desc(smem_u32(S.dout[0]), 16, 1024);
             const uint64_t qm0 = sw128_desc(smem_u32(S.q[0]), kHalfTile / 2, 1024);
             const uint64_t om0 = sw128_desc(smem_u32(S.dout[0]), kHalfTile / 2, 1024);
-            // S^T = K Q^T and dP^T = V dO^T of item n into buffer n & 1
-            auto issue_t = [&](int n) -> bool {
+            // S^T = K Q^T (issue_st) and dP^T = V dO^T (issue_dp) of item n into buffer n & 1
+            auto issue_st = [&](int n) -> bool {
                 const int s = n % kDkvStages;
-                const uint32_t buf = (uint32_t)(n & 1) * 64;
-                if (!mbar_wait(&S.full[s], (n / kDkvStages) & 1, abort, status)) return false;
+                if (!warp_wait(&S.full[s], (n / kDkvStages) & 1, abort, status)) return false;
                 tc_fence_after();
-                const uint64_t qd = desc_add(qk0, s * kHalfTile), od = desc_add(ok0, s * kHalfTile);
-                const uint32_t dst = tmem + cST + buf, ddp = tmem + cDP + buf;
+                const uint64_t qd = desc_add(qk0, s * kHalfTile);
+                const uint32_t dst = tmem + cST + (uint32_t)(n & 1) * 64;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint32_t offa = (kk >> 2) * (kTile / 2) + (kk & 3) * 32;
                     const uint32_t offb = (kk >> 2) * (kHalfTile / 2) + (kk & 3) * 32;
-                    mma_ss(dst, desc_add(kd, offa), desc_add(qd, offb), idT, kk > 0);
+                    if (leader) mma_ss(dst, desc_add(kd, offa), desc_add(qd, offb), idT, kk > 0);
                 }
-                mma_commit(&S.st_full[n & 1]);
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t offa = (kk >> 2) * (kTile / 2) + (kk & 3) * 32;
-                    const uint32_t offb = (kk >> 2) * (kHalfTile / 2) + (kk & 3) * 32;
-                    mma_ss(ddp, desc_add(vd, offa), desc_add(od, offb), idT, kk > 0);
-                }
-                mma_commit(&S.dp_full[n & 1]);
+                if (leader) mma_commit(&S.st_full[n & 1]);
                 return true;
             };
-            bool ok = mbar_wait(&S.kv_full, 0, abort, status) && issue_t(0) && (nw < 2 || issue_t(1));
+            auto issue_dp = [&](int n) {  // stage already waited for by issue_st(n)
+                const int s = n % kDkvStages;
+                const uint64_t od = desc_add(ok0, s * kHalfTile);
+                const uint32_t ddp = tmem + cDP + (uint32_t)(n & 1) * 64;
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t offa = (kk >> 2) * (kTile / 2) + (kk & 3) * 32;
+                    const uint32_t offb = (kk >> 2) * (kHalfTile / 2) + (kk & 3) * 32;
+                    if (leader) mma_ss(ddp, desc_add(vd, offa), desc_add(od, offb), idT, kk > 0);
+                }
+                if (leader) mma_commit(&S.dp_full[n & 1]);
+            };
+            bool ok = warp_wait(&S.kv_full, 0, abort, status) && issue_st(0);
+            if (ok) issue_dp(0);
+            if (ok && nw > 1) {
+                ok = issue_st(1);
+                if (ok) issue_dp(1);
+            }
+            // Per item n: dV(n), S^T(n+2), [dS^T(n) ready] dK(n), dP^T(n+2). Item n+2
+            // reuses item n's buffers; every MMA that reads them (dV(n) reads P^T
+            // from the S^T buffer, dK(n) reads dS^T from the dP^T buffer) is issued
+            // before the product that overwrites them, and MMAs run in order. S^T(n+2)
+            // goes ahead of the dS^T wait so the tensor core has work while it is formed.
             for (int n = 0; ok && n < nw; ++n) {
                 const int s = n % kDkvStages;
                 const uint32_t buf = (uint32_t)(n & 1) * 64;
                 const uint64_t qm = desc_add(qm0, s * kHalfTile), om = desc_add(om0, s * kHalfTile);
                 const uint32_t pa = tmem + cST + buf, sa = tmem + cDP + buf, acc = n > 0 ? 1u : 0u;
-                if (!mbar_wait(&S.p_ready[n & 1], (n >> 1) & 1, abort, status)) break;
+                if (!warp_wait(&S.p_ready[n & 1], (n >> 1) & 1, abort, status)) break;
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    mma_ts(tmem + cDV, pa + kk * 8, desc_add(om, kk * 2048), idMN, kk > 0 ? 1u : acc);
-                if (!mbar_wait(&S.ds_ready[n & 1], (n >> 1) & 1, abort, status)) break;
+                    if (leader) mma_ts(tmem + cDV, pa + kk * 8, desc_add(om, kk * 2048), idMN, kk > 0 ? 1u : acc);
+                if (n + 2 < nw && !issue_st(n + 2)) break;
+                if (!warp_wait(&S.ds_ready[n & 1], (n >> 1) & 1, abort, status)) break;
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    mma_ts(tmem + cDK, sa + kk * 8, desc_add(qm, kk * 2048), idMN, kk > 0 ? 1u : acc);
-                mma_commit(&S.empty[s]);
-                // the products of item n+2 reuse this buffer: the MMAs above, which
-                // read P^T and dS^T from it, were issued first and run in order
-                if (n + 2 < nw && !issue_t(n + 2)) break;
+                    if (leader) mma_ts(tmem + cDK, sa + kk * 8, desc_add(qm, kk * 2048), idMN, kk > 0 ? 1u : acc);
+                if (leader) mma_commit(&S.empty[s]);
+                if (n + 2 < nw) issue_dp(n + 2);
             }
-            mma_commit(&S.acc_done);
-            mma_commit(&S.fin);
+            if (leader) mma_commit(&S.acc_done);
+            if (leader) mma_commit(&S.fin);
             wait_done(&S.fin, 0);
         }
     } else {
@@ -479,7 +489,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             }
         }
     } else if (warp == 1) {
-        if (lane == 0 && nt > 0) {
+        if (nt > 0) {
+            const bool leader = elect_one();
             const uint32_t idKM = idesc_bf16(128, 128, false, false);
             const uint32_t idMN = idesc_bf16(128, 128, false, true);
             const uint64_t qd = sw128_desc(smem_u32(S.q), 16, 1024);
@@ -492,42 +503,42 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             const uint64_t km1 = sw128_desc(smem_u32(S.k[1]), kTile / 2, 1024);
             auto issue_s_dp = [&](int n) -> bool {
                 const int s = n & 1;
-                if (!mbar_wait(&S.full[s], (n >> 1) & 1, abort, status)) return false;
+                if (!warp_wait(&S.full[s], (n >> 1) & 1, abort, status)) return false;
                 const uint64_t kd = s ? kd1 : kd0, vd = s ? vd1 : vd0;
-                if (n > 0 && !mbar_wait(&S.s_free, (n - 1) & 1, abort, status)) return false;
+                if (n > 0 && !warp_wait(&S.s_free, (n - 1) & 1, abort, status)) return false;
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint32_t off = (kk >> 2) * (kTile / 2) + (kk & 3) * 32;
-                    mma_ss(tmem + cS, desc_add(qd, off), desc_add(kd, off), idKM, kk > 0);
+                    if (leader) mma_ss(tmem + cS, desc_add(qd, off), desc_add(kd, off), idKM, kk > 0);
                 }
-                mma_commit(&S.s_full);
-                if (n > 0 && !mbar_wait(&S.dp_free, (n - 1) & 1, abort, status)) return false;
+                if (leader) mma_commit(&S.s_full);
+                if (n > 0 && !warp_wait(&S.dp_free, (n - 1) & 1, abort, status)) return false;
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint32_t off = (kk >> 2) * (kTile / 2) + (kk & 3) * 32;
-                    mma_ss(tmem + cDP, desc_add(od, off), desc_add(vd, off), idKM, kk > 0);
+                    if (leader) mma_ss(tmem + cDP, desc_add(od, off), desc_add(vd, off), idKM, kk > 0);
                 }
-                mma_commit(&S.dp_full);
+                if (leader) mma_commit(&S.dp_full);
                 return true;
             };
-            bool ok = mbar_wait(&S.qo_full, 0, abort, status) && issue_s_dp(0);
+            bool ok = warp_wait(&S.qo_full, 0, abort, status) && issue_s_dp(0);
             for (int n = 0; ok && n < nt; ++n) {
                 const int s = n & 1;
                 if (n + 1 < nt && !issue_s_dp(n + 1)) break;
-                if (!mbar_wait(&S.ds_ready, n & 1, abort, status)) break;
+                if (!warp_wait(&S.ds_ready, n & 1, abort, status)) break;
                 tc_fence_after();
                 const uint64_t km = s ? km1 : km0;
                 const uint32_t sa = tmem + cDS + s * 64, acc = n > 0 ? 1u : 0u;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    mma_ts(tmem + cDQ, sa + kk * 8, desc_add(km, kk * 2048), idMN, kk > 0 ? 1u : acc);
-                mma_commit(&S.empty[s]);
-                mma_commit(&S.dq_done);
+                    if (leader) mma_ts(tmem + cDQ, sa + kk * 8, desc_add(km, kk * 2048), idMN, kk > 0 ? 1u : acc);
+                if (leader) mma_commit(&S.empty[s]);
+                if (leader) mma_commit(&S.dq_done);
             }
-            mma_commit(&S.acc_done);
-            mma_commit(&S.fin);
+            if (leader) mma_commit(&S.acc_done);
+            if (leader) mma_commit(&S.fin);
             wait_done(&S.fin, 0);
         }
     } else {

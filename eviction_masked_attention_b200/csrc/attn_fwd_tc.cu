@@ -108,7 +108,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             }
         }
     } else if (warp == 1) {
-        if (lane == 0 && nt > 0) {
+        if (nt > 0) {
+            const bool leader = elect_one();
             const uint32_t idS = idesc_bf16(128, 128, false, false);
             const uint32_t idPV = idesc_bf16(128, 128, false, true);
             const uint64_t qd = sw128_desc(smem_u32(S.q), 16, 1024);
@@ -116,39 +117,39 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             const uint64_t kd1 = sw128_desc(smem_u32(S.k[1]), 16, 1024);
             const uint64_t vd0 = sw128_desc(smem_u32(S.v[0]), kTileBytes / 2, 1024);
             const uint64_t vd1 = sw128_desc(smem_u32(S.v[1]), kTileBytes / 2, 1024);
-            bool ok = mbar_wait(&S.bar_q, 0, abort, status);
+            bool ok = warp_wait(&S.bar_q, 0, abort, status);
             auto issue_s = [&](int n) -> bool {
                 const int s = n & 1;
-                if (!mbar_wait(&S.kfull[s], (n >> 1) & 1, abort, status)) return false;
+                if (!warp_wait(&S.kfull[s], (n >> 1) & 1, abort, status)) return false;
                 tc_fence_after();
                 const uint64_t kd = s ? kd1 : kd0;
                 const uint32_t d = tmem + s * 128;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint32_t off = (kk >> 2) * (kTileBytes / 2) + (kk & 3) * 32;
-                    mma_ss(d, desc_add(qd, off), desc_add(kd, off), idS, kk > 0);
+                    if (leader) mma_ss(d, desc_add(qd, off), desc_add(kd, off), idS, kk > 0);
                 }
-                mma_commit(&S.kempty[s]);
-                mma_commit(&S.sfull[s]);
+                if (leader) mma_commit(&S.kempty[s]);
+                if (leader) mma_commit(&S.sfull[s]);
                 return true;
             };
             if (ok) ok = issue_s(0);
             for (int n = 0; ok && n < nt; ++n) {
                 const int s = n & 1;
                 if (n + 1 < nt && !issue_s(n + 1)) break;
-                if (!mbar_wait(&S.pfull[s], (n >> 1) & 1, abort, status)) break;
-                if (!mbar_wait(&S.vfull[s], (n >> 1) & 1, abort, status)) break;
+                if (!warp_wait(&S.pfull[s], (n >> 1) & 1, abort, status)) break;
+                if (!warp_wait(&S.vfull[s], (n >> 1) & 1, abort, status)) break;
                 tc_fence_after();
                 const uint64_t vd = s ? vd1 : vd0;
                 const uint32_t pa = tmem + s * 128, acc = n > 0 ? 1u : 0u;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    mma_ts(tmem + 256, pa + kk * 8, desc_add(vd, kk * 2048), idPV, kk > 0 ? 1u : acc);
-                mma_commit(&S.vempty[s]);
-                mma_commit(&S.odone);
+                    if (leader) mma_ts(tmem + 256, pa + kk * 8, desc_add(vd, kk * 2048), idPV, kk > 0 ? 1u : acc);
+                if (leader) mma_commit(&S.vempty[s]);
+                if (leader) mma_commit(&S.odone);
             }
             // all issued MMAs complete before TMEM can be released
-            mma_commit(&S.fin);
+            if (leader) mma_commit(&S.fin);
             wait_final(&S.fin, 0);
         }
     } else {
@@ -367,7 +368,8 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
             }
         }
     } else if (warp == 1) {
-        if (lane == 0 && nt > 0) {
+        if (nt > 0) {
+            const bool leader = elect_one();
             const uint32_t idS = idesc_bf16(128, 128, false, false);
             const uint32_t idPV = idesc_bf16(128, 128, false, true);
             const uint64_t qd0 = sw128_desc(smem_u32(S.q[0]), 16, 1024);
@@ -382,48 +384,48 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint32_t off = (kk >> 2) * (kTileBytes / 2) + (kk & 3) * 32;
-                    mma_ss(d, desc_add(qd, off), desc_add(kd, off), idS, kk > 0);
+                    if (leader) mma_ss(d, desc_add(qd, off), desc_add(kd, off), idS, kk > 0);
                 }
-                mma_commit(&S.sfull[x]);
+                if (leader) mma_commit(&S.sfull[x]);
             };
             auto issue_pv = [&](int x, int n) {
                 const uint64_t vd = (n & 1) ? vd1 : vd0;
                 const uint32_t d = tmem + 256 + x * 128, pa = tmem + x * 128, acc = n > 0 ? 1u : 0u;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    mma_ts(d, pa + kk * 8, desc_add(vd, kk * 2048), idPV, kk > 0 ? 1u : acc);
-                mma_commit(&S.odone[x]);
+                    if (leader) mma_ts(d, pa + kk * 8, desc_add(vd, kk * 2048), idPV, kk > 0 ? 1u : acc);
+                if (leader) mma_commit(&S.odone[x]);
             };
-            bool ok = mbar_wait(&S.bar_q, 0, abort, status) &&
-                      mbar_wait(&S.kfull[0], 0, abort, status);
+            bool ok = warp_wait(&S.bar_q, 0, abort, status) &&
+                      warp_wait(&S.kfull[0], 0, abort, status);
             if (ok) {
                 tc_fence_after();
                 issue_s(0, 0);
                 issue_s(1, 0);
-                mma_commit(&S.kempty[0]);
+                if (leader) mma_commit(&S.kempty[0]);
             }
             for (int n = 0; ok && n < nt; ++n) {
                 const int s = n & 1;
                 const bool more = n + 1 < nt;
-                if (!mbar_wait(&S.pfull[0], n & 1, abort, status)) break;
-                if (!mbar_wait(&S.vfull[s], (n >> 1) & 1, abort, status)) break;
+                if (!warp_wait(&S.pfull[0], n & 1, abort, status)) break;
+                if (!warp_wait(&S.vfull[s], (n >> 1) & 1, abort, status)) break;
                 tc_fence_after();
                 issue_pv(0, n);
                 if (more) {
-                    if (!mbar_wait(&S.kfull[(n + 1) & 1], ((n + 1) >> 1) & 1, abort, status)) break;
+                    if (!warp_wait(&S.kfull[(n + 1) & 1], ((n + 1) >> 1) & 1, abort, status)) break;
                     tc_fence_after();
                     issue_s(0, n + 1);
                 }
-                if (!mbar_wait(&S.pfull[1], n & 1, abort, status)) break;
+                if (!warp_wait(&S.pfull[1], n & 1, abort, status)) break;
                 tc_fence_after();
                 issue_pv(1, n);
-                mma_commit(&S.vempty[s]);
+                if (leader) mma_commit(&S.vempty[s]);
                 if (more) {
                     issue_s(1, n + 1);
-                    mma_commit(&S.kempty[(n + 1) & 1]);
+                    if (leader) mma_commit(&S.kempty[(n + 1) & 1]);
                 }
             }
-            mma_commit(&S.fin);
+            if (leader) mma_commit(&S.fin);
             wait_final(&S.fin, 0);
         }
     } else {

@@ -156,6 +156,27 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
     }
 }
 
+// mbar_wait by every lane of a warp, with one verdict for the whole warp so
+// that its control flow stays converged.
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
+                                          int32_t *status) {
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, status));
+}
+
+// One lane of the (converged) warp. Tensor-core issue runs on the whole warp,
+// with only the elected lane issuing tcgen05 instructions: kept converged, the
+// issuing code stays on the uniform datapath and is not slowed by the other
+// warps of its scheduler.
+__device__ __forceinline__ bool elect_one() {
+    uint32_t pred = 0;
+    asm volatile(
+        "{\n\t.reg .pred P;\n\t"
+        "elect.sync _|P, 0xffffffff;\n\t"
+        "selp.b32 %0, 1, 0, P;\n\t}"
+        : "=r"(pred));
+    return pred != 0;
+}
+
 // True once some CTA of the grid recorded a timeout; kernels check it on entry.
 __device__ __forceinline__ bool grid_timed_out(const int32_t *status) {
     return status && *reinterpret_cast<const volatile int32_t *>(status) == KVS_ERR_TIMEOUT;
