@@ -414,7 +414,10 @@ struct DqSmem {
     uint8_t v[2][kTile];
     uint32_t bits[2][128 * 4];  // mask rows of the key tile in each stage (partial tiles)
     int32_t pid[2];             // its partial index (-1: full)
-    uint64_t qo_full, full[2], empty[2], s_full, dp_full, s_free, dp_free, ds_ready, dq_done,
+    // K (with the tile's mask rows) and V stages are released separately: V after
+    // dP, K only after dQ, so the next V load is not held back by the dS phase
+    uint64_t qo_full, kfull[2], kempty[2], vfull[2], vempty[2], s_full, dp_full, s_free, dp_free,
+        ds_ready, dq_done,
         acc_done, fin;
     uint32_t tmem_base;
     int abort;
@@ -442,8 +445,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     if (threadIdx.x == 0) {
         mbar_init(&S.qo_full, 1);
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&S.full[i], 1);
-            mbar_init(&S.empty[i], 1);
+            mbar_init(&S.kfull[i], 1);
+            mbar_init(&S.kempty[i], 1);
+            mbar_init(&S.vfull[i], 1);
+            mbar_init(&S.vempty[i], 1);
         }
         mbar_init(&S.s_full, 1);
         mbar_init(&S.dp_full, 1);
@@ -476,16 +481,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             tma_load_4d(S.dout + kTile / 2, &tmO, &S.qo_full, 64, hq, q0, b);
             for (int n = 0; n < nt; ++n) {
                 const int s = n & 1;
-                if (n >= 2 && !mbar_wait(&S.empty[s], ((n >> 1) - 1) & 1, abort, status)) break;
                 const int k0 = m.row_col[e0 + n] * 128;
+                if (n >= 2 && !mbar_wait(&S.kempty[s], ((n >> 1) - 1) & 1, abort, status)) break;
                 const int32_t pid = m.row_pidx[e0 + n];
                 S.pid[s] = pid;
-                mbar_expect_tx(&S.full[s], 2 * kTile + (pid >= 0 ? 2048u : 0u));
-                tma_load_4d(S.k[s], &tmK, &S.full[s], 0, kvh, k0, b);
-                tma_load_4d(S.k[s] + kTile / 2, &tmK, &S.full[s], 64, kvh, k0, b);
-                tma_load_4d(S.v[s], &tmV, &S.full[s], 0, kvh, k0, b);
-                tma_load_4d(S.v[s] + kTile / 2, &tmV, &S.full[s], 64, kvh, k0, b);
-                if (pid >= 0) bulk_load(S.bits[s], m.bits + (int64_t)pid * 512, 2048, &S.full[s]);
+                mbar_expect_tx(&S.kfull[s], kTile + (pid >= 0 ? 2048u : 0u));
+                tma_load_4d(S.k[s], &tmK, &S.kfull[s], 0, kvh, k0, b);
+                tma_load_4d(S.k[s] + kTile / 2, &tmK, &S.kfull[s], 64, kvh, k0, b);
+                if (pid >= 0) bulk_load(S.bits[s], m.bits + (int64_t)pid * 512, 2048, &S.kfull[s]);
+                if (n >= 2 && !mbar_wait(&S.vempty[s], ((n >> 1) - 1) & 1, abort, status)) break;
+                mbar_expect_tx(&S.vfull[s], kTile);
+                tma_load_4d(S.v[s], &tmV, &S.vfull[s], 0, kvh, k0, b);
+                tma_load_4d(S.v[s] + kTile / 2, &tmV, &S.vfull[s], 64, kvh, k0, b);
             }
         }
     } else if (warp == 1) {
@@ -503,7 +510,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             const uint64_t km1 = sw128_desc(smem_u32(S.k[1]), kTile / 2, 1024);
             auto issue_s_dp = [&](int n) -> bool {
                 const int s = n & 1;
-                if (!warp_wait(&S.full[s], (n >> 1) & 1, abort, status)) return false;
+                if (!warp_wait(&S.kfull[s], (n >> 1) & 1, abort, status)) return false;
                 const uint64_t kd = s ? kd1 : kd0, vd = s ? vd1 : vd0;
                 if (n > 0 && !warp_wait(&S.s_free, (n - 1) & 1, abort, status)) return false;
                 tc_fence_after();
@@ -514,6 +521,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 }
                 if (leader) mma_commit(&S.s_full);
                 if (n > 0 && !warp_wait(&S.dp_free, (n - 1) & 1, abort, status)) return false;
+                if (!warp_wait(&S.vfull[s], (n >> 1) & 1, abort, status)) return false;
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
@@ -521,6 +529,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     if (leader) mma_ss(tmem + cDP, desc_add(od, off), desc_add(vd, off), idKM, kk > 0);
                 }
                 if (leader) mma_commit(&S.dp_full);
+                if (leader) mma_commit(&S.vempty[s]);
                 return true;
             };
             bool ok = warp_wait(&S.qo_full, 0, abort, status) && issue_s_dp(0);
@@ -534,7 +543,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
                     if (leader) mma_ts(tmem + cDQ, sa + kk * 8, desc_add(km, kk * 2048), idMN, kk > 0 ? 1u : acc);
-                if (leader) mma_commit(&S.empty[s]);
+                if (leader) mma_commit(&S.kempty[s]);
                 if (leader) mma_commit(&S.dq_done);
             }
             if (leader) mma_commit(&S.acc_done);
@@ -558,8 +567,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 break;
             }
             tc_fence_after();
-            // S_n complete implies stage s (K, V and the tile's mask rows) has
-            // landed; it is refilled only after dQ_n, i.e. after this item's dS
+            // the K stage carries the tile's mask rows; it is refilled only after
+            // dQ_n, i.e. after this item's dS
+            if (!warp_wait(&S.kfull[s], (n >> 1) & 1, abort, status)) {
+                ok = false;
+                break;
+            }
             const bool partial = S.pid[s] >= 0;  // same for the whole CTA
             uint2 bits = make_uint2(~0u, ~0u);
             if (partial) bits = *reinterpret_cast<const uint2 *>(&S.bits[s][row * 4 + half * 2]);
