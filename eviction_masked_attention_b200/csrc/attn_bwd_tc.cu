@@ -407,18 +407,21 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 // the next key tile are issued as soon as the elementwise warps have read the
 // current ones, so the tensor core computes them while dS is being formed.
 
+// K is needed from S_n until dQ_n, at the end of the item, V only for dP_n. K
+// therefore has three stages (the load of K_{n+1} overlaps item n instead of
+// waiting for dQ_{n-1}), V one: V_{n+1} loads while the elementwise warps form
+// P_n, long before dP_{n+1} is issued.
+constexpr int kDqKStages = 3;
+
 struct DqSmem {
     uint8_t q[kTile];
     uint8_t dout[kTile];
-    uint8_t k[2][kTile];
-    uint8_t v[2][kTile];
-    uint32_t bits[2][128 * 4];  // mask rows of the key tile in each stage (partial tiles)
-    int32_t pid[2];             // its partial index (-1: full)
-    // K (with the tile's mask rows) and V stages are released separately: V after
-    // dP, K only after dQ, so the next V load is not held back by the dS phase
-    uint64_t qo_full, kfull[2], kempty[2], vfull[2], vempty[2], s_full, dp_full, s_free, dp_free,
-        ds_ready, dq_done,
-        acc_done, fin;
+    uint8_t k[kDqKStages][kTile];
+    uint8_t v[kTile];
+    uint32_t bits[kDqKStages][128 * 4];  // mask rows of the key tile in each K stage (partial tiles)
+    int32_t pid[kDqKStages];             // its partial index (-1: full)
+    uint64_t qo_full, kfull[kDqKStages], kempty[kDqKStages], vfull, vempty, s_full, dp_full, s_free,
+        dp_free, ds_ready, dq_done, acc_done, fin;
     uint32_t tmem_base;
     int abort;
 };
@@ -444,12 +447,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
     if (threadIdx.x == 0) {
         mbar_init(&S.qo_full, 1);
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < kDqKStages; ++i) {
             mbar_init(&S.kfull[i], 1);
             mbar_init(&S.kempty[i], 1);
-            mbar_init(&S.vfull[i], 1);
-            mbar_init(&S.vempty[i], 1);
         }
+        mbar_init(&S.vfull, 1);
+        mbar_init(&S.vempty, 1);
         mbar_init(&S.s_full, 1);
         mbar_init(&S.dp_full, 1);
         mbar_init(&S.s_free, 256);
@@ -480,19 +483,21 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             tma_load_4d(S.dout, &tmO, &S.qo_full, 0, hq, q0, b);
             tma_load_4d(S.dout + kTile / 2, &tmO, &S.qo_full, 64, hq, q0, b);
             for (int n = 0; n < nt; ++n) {
-                const int s = n & 1;
+                const int ks = n % kDqKStages;
                 const int k0 = m.row_col[e0 + n] * 128;
-                if (n >= 2 && !mbar_wait(&S.kempty[s], ((n >> 1) - 1) & 1, abort, status)) break;
+                if (n >= kDqKStages &&
+                    !mbar_wait(&S.kempty[ks], ((n / kDqKStages) - 1) & 1, abort, status))
+                    break;
                 const int32_t pid = m.row_pidx[e0 + n];
-                S.pid[s] = pid;
-                mbar_expect_tx(&S.kfull[s], kTile + (pid >= 0 ? 2048u : 0u));
-                tma_load_4d(S.k[s], &tmK, &S.kfull[s], 0, kvh, k0, b);
-                tma_load_4d(S.k[s] + kTile / 2, &tmK, &S.kfull[s], 64, kvh, k0, b);
-                if (pid >= 0) bulk_load(S.bits[s], m.bits + (int64_t)pid * 512, 2048, &S.kfull[s]);
-                if (n >= 2 && !mbar_wait(&S.vempty[s], ((n >> 1) - 1) & 1, abort, status)) break;
-                mbar_expect_tx(&S.vfull[s], kTile);
-                tma_load_4d(S.v[s], &tmV, &S.vfull[s], 0, kvh, k0, b);
-                tma_load_4d(S.v[s] + kTile / 2, &tmV, &S.vfull[s], 64, kvh, k0, b);
+                S.pid[ks] = pid;
+                mbar_expect_tx(&S.kfull[ks], kTile + (pid >= 0 ? 2048u : 0u));
+                tma_load_4d(S.k[ks], &tmK, &S.kfull[ks], 0, kvh, k0, b);
+                tma_load_4d(S.k[ks] + kTile / 2, &tmK, &S.kfull[ks], 64, kvh, k0, b);
+                if (pid >= 0) bulk_load(S.bits[ks], m.bits + (int64_t)pid * 512, 2048, &S.kfull[ks]);
+                if (n >= 1 && !mbar_wait(&S.vempty, (n - 1) & 1, abort, status)) break;
+                mbar_expect_tx(&S.vfull, kTile);
+                tma_load_4d(S.v, &tmV, &S.vfull, 0, kvh, k0, b);
+                tma_load_4d(S.v + kTile / 2, &tmV, &S.vfull, 64, kvh, k0, b);
             }
         }
     } else if (warp == 1) {
@@ -502,16 +507,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             const uint32_t idMN = idesc_bf16(128, 128, false, true);
             const uint64_t qd = sw128_desc(smem_u32(S.q), 16, 1024);
             const uint64_t od = sw128_desc(smem_u32(S.dout), 16, 1024);
-            const uint64_t kd0 = sw128_desc(smem_u32(S.k[0]), 16, 1024);
-            const uint64_t kd1 = sw128_desc(smem_u32(S.k[1]), 16, 1024);
-            const uint64_t vd0 = sw128_desc(smem_u32(S.v[0]), 16, 1024);
-            const uint64_t vd1 = sw128_desc(smem_u32(S.v[1]), 16, 1024);
-            const uint64_t km0 = sw128_desc(smem_u32(S.k[0]), kTile / 2, 1024);
-            const uint64_t km1 = sw128_desc(smem_u32(S.k[1]), kTile / 2, 1024);
+            const uint64_t kd0 = sw128_desc(smem_u32(S.k[0]), 16, 1024);         // + stage * kTile
+            const uint64_t km0 = sw128_desc(smem_u32(S.k[0]), kTile / 2, 1024);  // MN-major view
+            const uint64_t vd = sw128_desc(smem_u32(S.v), 16, 1024);
             auto issue_s_dp = [&](int n) -> bool {
-                const int s = n & 1;
-                if (!warp_wait(&S.kfull[s], (n >> 1) & 1, abort, status)) return false;
-                const uint64_t kd = s ? kd1 : kd0, vd = s ? vd1 : vd0;
+                const int ks = n % kDqKStages;
+                if (!warp_wait(&S.kfull[ks], (n / kDqKStages) & 1, abort, status)) return false;
+                const uint64_t kd = desc_add(kd0, ks * kTile);
                 if (n > 0 && !warp_wait(&S.s_free, (n - 1) & 1, abort, status)) return false;
                 tc_fence_after();
 #pragma unroll
@@ -521,7 +523,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 }
                 if (leader) mma_commit(&S.s_full);
                 if (n > 0 && !warp_wait(&S.dp_free, (n - 1) & 1, abort, status)) return false;
-                if (!warp_wait(&S.vfull[s], (n >> 1) & 1, abort, status)) return false;
+                if (!warp_wait(&S.vfull, n & 1, abort, status)) return false;
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
@@ -529,7 +531,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     if (leader) mma_ss(tmem + cDP, desc_add(od, off), desc_add(vd, off), idKM, kk > 0);
                 }
                 if (leader) mma_commit(&S.dp_full);
-                if (leader) mma_commit(&S.vempty[s]);
+                if (leader) mma_commit(&S.vempty);
                 return true;
             };
             bool ok = warp_wait(&S.qo_full, 0, abort, status) && issue_s_dp(0);
@@ -538,12 +540,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 if (n + 1 < nt && !issue_s_dp(n + 1)) break;
                 if (!warp_wait(&S.ds_ready, n & 1, abort, status)) break;
                 tc_fence_after();
-                const uint64_t km = s ? km1 : km0;
+                const uint64_t km = desc_add(km0, (n % kDqKStages) * kTile);
                 const uint32_t sa = tmem + cDS + s * 64, acc = n > 0 ? 1u : 0u;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
                     if (leader) mma_ts(tmem + cDQ, sa + kk * 8, desc_add(km, kk * 2048), idMN, kk > 0 ? 1u : acc);
-                if (leader) mma_commit(&S.kempty[s]);
+                if (leader) mma_commit(&S.kempty[n % kDqKStages]);
                 if (leader) mma_commit(&S.dq_done);
             }
             if (leader) mma_commit(&S.acc_done);
@@ -569,13 +571,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             tc_fence_after();
             // the K stage carries the tile's mask rows; it is refilled only after
             // dQ_n, i.e. after this item's dS
-            if (!warp_wait(&S.kfull[s], (n >> 1) & 1, abort, status)) {
+            const int ks = n % kDqKStages;
+            if (!warp_wait(&S.kfull[ks], (n / kDqKStages) & 1, abort, status)) {
                 ok = false;
                 break;
             }
-            const bool partial = S.pid[s] >= 0;  // same for the whole CTA
+            const bool partial = S.pid[ks] >= 0;  // same for the whole CTA
             uint2 bits = make_uint2(~0u, ~0u);
-            if (partial) bits = *reinterpret_cast<const uint2 *>(&S.bits[s][row * 4 + half * 2]);
+            if (partial) bits = *reinterpret_cast<const uint2 *>(&S.bits[ks][row * 4 + half * 2]);
             // P = 2^(S c - LSE log2 e) for this thread's 64 key columns, kept as bf16
             // pairs; dS = P (dP - D) then rounds to bf16 for the dQ MMA
             uint32_t pp[32];
