@@ -472,7 +472,7 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
                 } else {
 #pragma unroll
                     for (int j = 0; j < 32; ++j)
-                        mx8[j & 7] = fmaxf(mx8[j & 7], fmaxf(__uint_as_float(r0[j]), __uint_as_float(r1[j])));
+                        mx8[j & 7] = max3f(mx8[j & 7], __uint_as_float(r0[j]), __uint_as_float(r1[j]));
                 }
             }
             float mraw = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
@@ -510,9 +510,9 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
             // columns overwrite the first of them). Half of the exponentials run on
             // the FMA pipe (exp2_fma), half on the special-function unit.
             const float nref = m_run == -INFINITY ? 0.f : -m_run;
-            float ls8[8];
+            uint64_t lsum2[4];  // four f32x2 partial row sums
 #pragma unroll
-            for (int u = 0; u < 8; ++u) ls8[u] = 0.f;
+            for (int u = 0; u < 4; ++u) lsum2[u] = 0ull;
 #pragma unroll 1
             for (int hc = 0; hc < 2; ++hc) {
                 uint32_t r0[32], r1[32], pk[32];
@@ -525,23 +525,31 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
                     const uint32_t(&r)[32] = cc ? r1 : r0;
                     const uint32_t w = cc ? w1 : w0;
 #pragma unroll
-                    for (int j = 0; j < 32; j += 2) {
-                        float x0, x1;
+                    for (int j = 0; j < 32; j += 4) {
+                        float x0, x1, x2, x3, p0, p1;
                         fma2(__uint_as_float(r[j]), __uint_as_float(r[j + 1]), scale_log2, nref, x0, x1);
-                        float p0 = exp2_fma(x0);
-                        float p1 = ex2(x1);
+                        fma2(__uint_as_float(r[j + 2]), __uint_as_float(r[j + 3]), scale_log2, nref, x2, x3);
+                        exp2_fma_x2(x0, x1, p0, p1);
+                        float p2 = ex2(x2), p3 = ex2(x3);
                         if (partial) {
                             p0 = ((w >> j) & 1u) ? p0 : 0.f;
                             p1 = ((w >> (j + 1)) & 1u) ? p1 : 0.f;
+                            p2 = ((w >> (j + 2)) & 1u) ? p2 : 0.f;
+                            p3 = ((w >> (j + 3)) & 1u) ? p3 : 0.f;
                         }
-                        ls8[(j >> 1) & 7] += p0 + p1;
+                        const int a = ((j >> 2) & 1) * 2;
+                        lsum2[a] = f2_add(lsum2[a], f2_make(p0, p1));
+                        lsum2[a + 1] = f2_add(lsum2[a + 1], f2_make(p2, p3));
                         pk[cc * 16 + (j >> 1)] = pack_bf16(p0, p1);
+                        pk[cc * 16 + (j >> 1) + 1] = pack_bf16(p2, p3);
                     }
                 }
                 tmem_st32(tmem + lane_off + cS + hc * 32, pk);
             }
-            const float lsum = ((ls8[0] + ls8[1]) + (ls8[2] + ls8[3])) + ((ls8[4] + ls8[5]) + (ls8[6] + ls8[7]));
-            l_run += lsum;
+            float ls[8];
+            f2_split(f2_add(lsum2[0], lsum2[2]), ls[0], ls[1]);
+            f2_split(f2_add(lsum2[1], lsum2[3]), ls[2], ls[3]);
+            l_run += (ls[0] + ls[1]) + (ls[2] + ls[3]);
             tmem_st_wait();
             tc_fence_before();
             mbar_arrive(&S.pfull[x]);

@@ -60,6 +60,57 @@ __device__ __forceinline__ float exp2_fma(float x) {
     return __uint_as_float(__float_as_uint(t) * 8388608u + __float_as_uint(p));
 }
 
+// Pairs of fp32 lanes in one 64-bit register, for the sm_100 f32x2 instructions
+// (one issue slot for two IEEE-rounded operations).
+__device__ __forceinline__ uint64_t f2_make(float a, float b) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+__device__ __forceinline__ void f2_split(uint64_t r, float &a, float &b) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r));
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
+// exp2_fma on two lanes with f32x2 arithmetic: the same operations, rounded the
+// same way per lane, in about half the issue slots.
+__device__ __forceinline__ void exp2_fma_x2(float x0, float x1, float &y0, float &y1) {
+    const uint64_t x = f2_make(fmaxf(x0, -127.f), fmaxf(x1, -127.f));
+    const uint64_t magic = f2_make(12582912.f, 12582912.f);
+    const uint64_t t = f2_add(x, magic);
+    const uint64_t f = f2_sub(x, f2_sub(t, magic));
+    uint64_t p = f2_fma(f2_make(5.517166907e-02f, 5.517166907e-02f), f,
+                        f2_make(2.426111222e-01f, 2.426111222e-01f));
+    p = f2_fma(p, f, f2_make(6.932609855e-01f, 6.932609855e-01f));
+    p = f2_fma(p, f, f2_make(9.999280735e-01f, 9.999280735e-01f));
+    float t0, t1, p0, p1;
+    f2_split(t, t0, t1);
+    f2_split(p, p0, p1);
+    y0 = __uint_as_float(__float_as_uint(t0) * 8388608u + __float_as_uint(p0));
+    y1 = __uint_as_float(__float_as_uint(t1) * 8388608u + __float_as_uint(p1));
+}
+
+// max(a, b, c) in one instruction.
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
 // Two fp32 lanes at once: (a0, a1) * (b, b) + (c, c).
 __device__ __forceinline__ void fma2(float a0, float a1, float b, float c, float &d0, float &d1) {
     uint64_t av, bv, cv, dv;
