@@ -36,17 +36,18 @@ __device__ __forceinline__ bool wait_done(uint64_t *bar, uint32_t parity) {
 }
 
 
-// D[b][h][t] = <dO, O>, L2[b][h][t] = lse * log2(e); rows t >= N get 0. Tpad = T*128.
+// D[b][h][t] = <dO, O>, NL2[b][h][t] = -lse * log2(e) (so that the exponent of P is one
+// fma of the raw score); rows t >= N get 0. Tpad = T*128.
 // O is o_hi (+ o_lo when the forward kept the rounding residual of its output).
 __global__ void k_bwd_prep(const __nv_bfloat16 *__restrict__ o, const __nv_bfloat16 *__restrict__ o_lo,
                            const __nv_bfloat16 *__restrict__ dO, const float *__restrict__ lse,
                            int32_t B, int32_t N, int32_t Hq, int32_t Tpad, float *__restrict__ Drow,
-                           float *__restrict__ L2) {
+                           float *__restrict__ NL2) {
     const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (row >= (int64_t)B * Hq * Tpad) return;
     const int64_t t = row % Tpad, bh = row / Tpad, h = bh % Hq, b = bh / Hq;
-    float s = 0.f, l2 = 0.f;
+    float s = 0.f, nl2 = 0.f;
     if (t < N) {
         const int64_t off = ((b * N + t) * Hq + h) * 128 + lane * 4;
         const uint2 a = *reinterpret_cast<const uint2 *>(o + off);
@@ -58,11 +59,11 @@ __global__ void k_bwd_prep(const __nv_bfloat16 *__restrict__ o, const __nv_bfloa
         }
         s = o0 * bf16_lo(c.x) + o1 * bf16_hi(c.x) + o2 * bf16_lo(c.y) + o3 * bf16_hi(c.y);
         for (int k = 16; k; k >>= 1) s += __shfl_xor_sync(0xffffffffu, s, k);
-        l2 = lse[(b * Hq + h) * N + t] * 1.4426950408889634f;
+        nl2 = -lse[(b * Hq + h) * N + t] * 1.4426950408889634f;
     }
     if (lane == 0) {
         Drow[row] = s;
-        L2[row] = l2;
+        NL2[row] = nl2;
     }
 }
 
@@ -107,7 +108,7 @@ struct DkvSmem {
     uint8_t v[kTile];
     uint8_t q[kDkvStages][kHalfTile];
     uint8_t dout[kDkvStages][kHalfTile];
-    float l2[kDkvStages][64];
+    float nl2[kDkvStages][64];  // -lse log2(e) of the half-tile rows
     float dd[kDkvStages][64];
     int32_t q0[kDkvStages], full_tile[kDkvStages];  // half-tile origin, FULL flag of its tile
     uint64_t kv_full, full[kDkvStages], empty[kDkvStages], st_full[2], dp_full[2], p_ready[2],
@@ -120,7 +121,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     k_attn_dkdv_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                    kvs_tile_mask m, int32_t Hq, int32_t Hkv, float scale, float scale_log2,
-                   const float *__restrict__ Drow, const float *__restrict__ L2,
+                   const float *__restrict__ Drow, const float *__restrict__ NL2,
                    __nv_bfloat16 *__restrict__ dk, __nv_bfloat16 *__restrict__ dv, int32_t *status) {
     extern __shared__ uint8_t smem_raw[];
     DkvSmem &S = *reinterpret_cast<DkvSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -187,7 +188,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 tma_load_4d(S.dout[s], &tmO, &S.full[s], 0, h, q0, b);
                 tma_load_4d(S.dout[s] + kHalfTile / 2, &tmO, &S.full[s], 64, h, q0, b);
                 const int64_t ro = ((int64_t)b * Hq + h) * Tpad + q0;
-                bulk_load(S.l2[s], L2 + ro, 256, &S.full[s]);
+                bulk_load(S.nl2[s], NL2 + ro, 256, &S.full[s]);
                 bulk_load(S.dd[s], Drow + ro, 256, &S.full[s]);
             }
         }
@@ -306,7 +307,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 tmem_ld32(tmem + lane_off + colS, r0);
                 tmem_ld32(tmem + lane_off + colS + 32, r1);
                 tmem_ld_wait();
-                const float4 *l2v = reinterpret_cast<const float4 *>(S.l2[s]);
+                const float4 *l2v = reinterpret_cast<const float4 *>(S.nl2[s]);
                 const bool all_vis = rlo <= 0 && rhi >= 64;
                 if (__all_sync(0xffffffffu, all_vis)) {
 #pragma unroll
@@ -317,8 +318,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                         const float a1 = __uint_as_float(rr < 32 ? r0[rr + 1] : r1[rr - 31]);
                         const float a2 = __uint_as_float(rr < 32 ? r0[rr + 2] : r1[rr - 30]);
                         const float a3 = __uint_as_float(rr < 32 ? r0[rr + 3] : r1[rr - 29]);
-                        pk[2 * i] = pack_bf16(ex2(fmaf(a0, scale_log2, -lv.x)), ex2(fmaf(a1, scale_log2, -lv.y)));
-                        pk[2 * i + 1] = pack_bf16(ex2(fmaf(a2, scale_log2, -lv.z)), ex2(fmaf(a3, scale_log2, -lv.w)));
+                        // half of the exponentials on the FMA pipe, half on the SFU
+                        float x0, x1, x2, x3, e0, e1;
+                        fma2v(a0, a1, scale_log2, lv.x, lv.y, x0, x1);
+                        fma2v(a2, a3, scale_log2, lv.z, lv.w, x2, x3);
+                        exp2_fma_x2(x0, x1, e0, e1);
+                        pk[2 * i] = pack_bf16(e0, e1);
+                        pk[2 * i + 1] = pack_bf16(ex2(x2), ex2(x3));
                     }
                 } else {
 #pragma unroll
@@ -330,7 +336,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                         for (int u = 0; u < 4; ++u) {
                             const int rr = 4 * i + u;
                             const float a = __uint_as_float(rr < 32 ? r0[rr] : r1[rr - 32]);
-                            q4[u] = (rr >= rlo && rr < rhi) ? ex2(fmaf(a, scale_log2, -ls[u])) : 0.f;
+                            q4[u] = (rr >= rlo && rr < rhi) ? ex2(fmaf(a, scale_log2, ls[u])) : 0.f;
                         }
                         pk[2 * i] = pack_bf16(q4[0], q4[1]);
                         pk[2 * i + 1] = pack_bf16(q4[2], q4[3]);
@@ -361,9 +367,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     const float a1 = __uint_as_float(rr < 32 ? r0[rr + 1] : r1[rr - 31]);
                     const float a2 = __uint_as_float(rr < 32 ? r0[rr + 2] : r1[rr - 30]);
                     const float a3 = __uint_as_float(rr < 32 ? r0[rr + 3] : r1[rr - 29]);
-                    dk2[2 * i] = pack_bf16(bf16_lo(pk[2 * i]) * (a0 - dv4.x), bf16_hi(pk[2 * i]) * (a1 - dv4.y));
-                    dk2[2 * i + 1] =
-                        pack_bf16(bf16_lo(pk[2 * i + 1]) * (a2 - dv4.z), bf16_hi(pk[2 * i + 1]) * (a3 - dv4.w));
+                    float d0, d1, d2, d3;
+                    f2_split(f2_mul(f2_make(bf16_lo(pk[2 * i]), bf16_hi(pk[2 * i])),
+                                    f2_sub(f2_make(a0, a1), f2_make(dv4.x, dv4.y))), d0, d1);
+                    f2_split(f2_mul(f2_make(bf16_lo(pk[2 * i + 1]), bf16_hi(pk[2 * i + 1])),
+                                    f2_sub(f2_make(a2, a3), f2_make(dv4.z, dv4.w))), d2, d3);
+                    dk2[2 * i] = pack_bf16(d0, d1);
+                    dk2[2 * i + 1] = pack_bf16(d2, d3);
                 }
                 tmem_st32(tmem + lane_off + colP, dk2);
             }
@@ -430,7 +440,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     k_attn_dq_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                  kvs_tile_mask m, int32_t Hq, int32_t Hkv, float scale, float scale_log2,
-                 const float *__restrict__ Drow, const float *__restrict__ L2,
+                 const float *__restrict__ Drow, const float *__restrict__ NL2,
                  __nv_bfloat16 *__restrict__ dq, int32_t *status) {
     extern __shared__ uint8_t smem_raw[];
     DqSmem &S = *reinterpret_cast<DqSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -560,7 +570,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
         const uint32_t col0 = half * 64;
         const int64_t ro = ((int64_t)b * Hq + hq) * Tpad + t;
-        const float l2 = L2[ro], dd = Drow[ro];
+        const float nl2 = NL2[ro], dd = Drow[ro];
+        const uint64_t dd2 = f2_make(dd, dd);
         bool ok = true;
         for (int n = 0; n < nt; ++n) {
             const int s = n & 1;
@@ -592,18 +603,22 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 if (!partial) {
 #pragma unroll
                     for (int jj = 0; jj < 32; jj += 2) {
-                        pp[jj >> 1] = pack_bf16(ex2(fmaf(__uint_as_float(r0[jj]), scale_log2, -l2)),
-                                                ex2(fmaf(__uint_as_float(r0[jj + 1]), scale_log2, -l2)));
-                        pp[16 + (jj >> 1)] = pack_bf16(ex2(fmaf(__uint_as_float(r1[jj]), scale_log2, -l2)),
-                                                       ex2(fmaf(__uint_as_float(r1[jj + 1]), scale_log2, -l2)));
+                        // first 32 columns on the FMA pipe, last 32 on the SFU
+                        float x0, x1, x2, x3, e0, e1;
+                        fma2(__uint_as_float(r0[jj]), __uint_as_float(r0[jj + 1]), scale_log2, nl2, x0, x1);
+                        fma2(__uint_as_float(r1[jj]), __uint_as_float(r1[jj + 1]), scale_log2, nl2, x2, x3);
+                        exp2_fma_x2(x0, x1, e0, e1);
+                        pp[jj >> 1] = pack_bf16(e0, e1);
+                        pp[16 + (jj >> 1)] = pack_bf16(ex2(x2), ex2(x3));
                     }
                 } else {
 #pragma unroll
                     for (int jj = 0; jj < 32; jj += 2) {
-                        const float e0 = ex2(fmaf(__uint_as_float(r0[jj]), scale_log2, -l2));
-                        const float e1 = ex2(fmaf(__uint_as_float(r0[jj + 1]), scale_log2, -l2));
-                        const float e2 = ex2(fmaf(__uint_as_float(r1[jj]), scale_log2, -l2));
-                        const float e3 = ex2(fmaf(__uint_as_float(r1[jj + 1]), scale_log2, -l2));
+                        float x0, x1, x2, x3, e0, e1;
+                        fma2(__uint_as_float(r0[jj]), __uint_as_float(r0[jj + 1]), scale_log2, nl2, x0, x1);
+                        fma2(__uint_as_float(r1[jj]), __uint_as_float(r1[jj + 1]), scale_log2, nl2, x2, x3);
+                        exp2_fma_x2(x0, x1, e0, e1);
+                        const float e2 = ex2(x2), e3 = ex2(x3);
                         pp[jj >> 1] = pack_bf16(((bits.x >> jj) & 1u) ? e0 : 0.f,
                                                 ((bits.x >> (jj + 1)) & 1u) ? e1 : 0.f);
                         pp[16 + (jj >> 1)] = pack_bf16(((bits.y >> jj) & 1u) ? e2 : 0.f,
@@ -626,10 +641,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 mbar_arrive(&S.dp_free);
 #pragma unroll
                 for (int jj = 0; jj < 32; jj += 2) {
-                    pk[jj >> 1] = pack_bf16(bf16_lo(pp[jj >> 1]) * (__uint_as_float(r0[jj]) - dd),
-                                            bf16_hi(pp[jj >> 1]) * (__uint_as_float(r0[jj + 1]) - dd));
-                    pk[16 + (jj >> 1)] = pack_bf16(bf16_lo(pp[16 + (jj >> 1)]) * (__uint_as_float(r1[jj]) - dd),
-                                                   bf16_hi(pp[16 + (jj >> 1)]) * (__uint_as_float(r1[jj + 1]) - dd));
+                    float d0, d1, d2, d3;
+                    const uint32_t pa = pp[jj >> 1], pb = pp[16 + (jj >> 1)];
+                    f2_split(f2_mul(f2_make(bf16_lo(pa), bf16_hi(pa)),
+                                    f2_sub(f2_make(__uint_as_float(r0[jj]), __uint_as_float(r0[jj + 1])), dd2)),
+                             d0, d1);
+                    f2_split(f2_mul(f2_make(bf16_lo(pb), bf16_hi(pb)),
+                                    f2_sub(f2_make(__uint_as_float(r1[jj]), __uint_as_float(r1[jj + 1])), dd2)),
+                             d2, d3);
+                    pk[jj >> 1] = pack_bf16(d0, d1);
+                    pk[16 + (jj >> 1)] = pack_bf16(d2, d3);
                 }
             }
             // dQ of item n-1 must be complete: its MMA has then consumed ds_ready
@@ -676,12 +697,12 @@ cudaError_t launch_bwd_tc(const void *q, const void *k, const void *v, const voi
     if (!*map_ok) return cudaSuccess;
     const int32_t Tpad = m.T * 128;
     float *Drow = (float *)ws;
-    float *L2 = Drow + (size_t)m.B * Hq * Tpad;
+    float *NL2 = Drow + (size_t)m.B * Hq * Tpad;
     const int64_t rows = (int64_t)m.B * Hq * Tpad;
     if (stages & KVS_BWD_PREP)
         k_bwd_prep<<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(
             (const __nv_bfloat16 *)o, (const __nv_bfloat16 *)o_lo, (const __nv_bfloat16 *)dO, lse,
-            m.B, m.N, Hq, Tpad, Drow, L2);
+            m.B, m.N, Hq, Tpad, Drow, NL2);
     const float sl2 = scale * 1.4426950408889634f;
     cudaError_t e = cudaSuccess;
     if (stages & KVS_BWD_DKDV) {
@@ -690,7 +711,7 @@ cudaError_t launch_bwd_tc(const void *q, const void *k, const void *v, const voi
                                  (int)smem);
         if (e != cudaSuccess) return e;
         k_attn_dkdv_tc<<<(unsigned)((int64_t)m.B * Hkv * m.T), kBwdThreads, smem, s>>>(
-            tq64, tk, tv, to64, m, Hq, Hkv, scale, sl2, Drow, L2, (__nv_bfloat16 *)dk,
+            tq64, tk, tv, to64, m, Hq, Hkv, scale, sl2, Drow, NL2, (__nv_bfloat16 *)dk,
             (__nv_bfloat16 *)dv, status);
     }
     if (stages & KVS_BWD_DQ) {
@@ -699,7 +720,7 @@ cudaError_t launch_bwd_tc(const void *q, const void *k, const void *v, const voi
                                  (int)smem);
         if (e != cudaSuccess) return e;
         k_attn_dq_tc<<<(unsigned)((int64_t)m.B * Hq * m.T), kBwdThreads, smem, s>>>(
-            tq, tk, tv, to, m, Hq, Hkv, scale, sl2, Drow, L2, (__nv_bfloat16 *)dq, status);
+            tq, tk, tv, to, m, Hq, Hkv, scale, sl2, Drow, NL2, (__nv_bfloat16 *)dq, status);
     }
     return cudaGetLastError();
 }
