@@ -9,7 +9,7 @@
 // Grid (split, kv head, sequence); one CTA streams a contiguous range of live
 // entries of one kv head for all G query heads that share it, so every K/V
 // byte is read from HBM once. Each of the 4 warps takes 16-entry chunks w,
-// w+4, ... and keeps a 3-stage ring of them in flight: its lanes copy the
+// w+4, ... and keeps a 2-stage ring of them in flight: its lanes copy the
 // 256-byte key and value rows (found through the block table slice held in
 // shared memory; a 16-token block is 16 consecutive rows, with 1-token blocks
 // every row comes from its own slot) in 16-byte cp.async pieces into rows of
@@ -27,7 +27,7 @@
 namespace kvs {
 
 constexpr int kDmWarps = 4;      // each warp streams and computes its own chunks
-constexpr int kDmStages = 3;     // ring depth per warp
+constexpr int kDmStages = 2;     // ring depth per warp (2: three CTAs fit on an SM)
 constexpr int kDmRow = 272;      // staged row stride in bytes (256 + 16)
 constexpr int kDmChunk = 16;     // entries per stage
 constexpr int kDmThreads = 32 * kDmWarps;
@@ -72,7 +72,10 @@ __device__ __forceinline__ void cp_async_wait() {
     asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-template <int G>
+// BS is the block size when it is one the workloads use (16: a chunk is one whole
+// block; 1: one block per entry), 0 for any other; it only shortens the address
+// arithmetic of the copies.
+template <int G, int BS>
 __global__ void __launch_bounds__(kDmThreads)
     k_decode_mma(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ kc,
                  const __nv_bfloat16 *__restrict__ vc, const int32_t *__restrict__ block_table,
@@ -117,15 +120,30 @@ __global__ void __launch_bounds__(kDmThreads)
             const int32_t t0 = t_begin + c * kDmChunk;
             const int nv = min(kDmChunk, t_end - t0);
             const uint32_t kd = smem_u32(S.k[w][s]) + piece * 16, vd = smem_u32(S.v[w][s]) + piece * 16;
+            if constexpr (BS == kDmChunk) {
+                // splits start at multiples of 128 entries, so a chunk is exactly one block
+                const int64_t base = (int64_t)S.blk[t0 / kDmChunk - blk0] * blk_stride + head_off + piece * 8;
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const int e = par + 2 * j;
-                if (e < nv) {
-                    const int32_t t = t0 + e;
-                    const int64_t off = (int64_t)S.blk[t / bs - blk0] * blk_stride + head_off +
-                                        (int64_t)(t % bs) * D + piece * 8;
-                    cp_async16(kd + e * kDmRow, kc + off);
-                    cp_async16(vd + e * kDmRow, vc + off);
+                for (int j = 0; j < 8; ++j) {
+                    const int e = par + 2 * j;
+                    if (e < nv) {
+                        cp_async16(kd + e * kDmRow, kc + base + e * D);
+                        cp_async16(vd + e * kDmRow, vc + base + e * D);
+                    }
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int e = par + 2 * j;
+                    if (e < nv) {
+                        const int32_t t = t0 + e;
+                        const int64_t off =
+                            BS == 1 ? (int64_t)S.blk[t - blk0] * blk_stride + head_off + piece * 8
+                                    : (int64_t)S.blk[t / bs - blk0] * blk_stride + head_off +
+                                          (int64_t)(t % bs) * D + piece * 8;
+                        cp_async16(kd + e * kDmRow, kc + off);
+                        cp_async16(vd + e * kDmRow, vc + off);
+                    }
                 }
             }
         }
@@ -276,17 +294,17 @@ __global__ void __launch_bounds__(kDmThreads)
 
 size_t decode_mma_smem() { return sizeof(DmSmem) + 128; }
 
-template <int G>
+template <int G, int BS>
 static cudaError_t launch_g(const void *q, const void *kc, const void *vc, const int32_t *bt,
                             const int32_t *nt, int32_t B, int32_t Hq, int32_t Hkv, int32_t bs,
                             int32_t max_blocks, float scale_log2, int32_t tps, int32_t max_splits,
                             void *o, float *partials, int32_t *status, cudaStream_t s) {
     const size_t smem = decode_mma_smem();
     cudaError_t e =
-        cudaFuncSetAttribute(k_decode_mma<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        cudaFuncSetAttribute(k_decode_mma<G, BS>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid(max_splits, Hkv, B);
-    k_decode_mma<G><<<grid, kDmThreads, smem, s>>>(
+    k_decode_mma<G, BS><<<grid, kDmThreads, smem, s>>>(
         (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)kc, (const __nv_bfloat16 *)vc, bt, nt, Hq,
         Hkv, bs, max_blocks, scale_log2, tps, max_splits, (__nv_bfloat16 *)o, partials, status);
     return cudaGetLastError();
@@ -297,15 +315,20 @@ cudaError_t launch_decode_mma(int G, const void *q, const void *kc, const void *
                               int32_t Hkv, int32_t bs, int32_t max_blocks, float scale_log2,
                               int32_t tps, int32_t max_splits, void *o, float *partials,
                               int32_t *status, cudaStream_t s) {
-#define KVS_DM(GG)                                                                               \
-    return launch_g<GG>(q, kc, vc, bt, nt, B, Hq, Hkv, bs, max_blocks, scale_log2, tps, max_splits, \
-                        o, partials, status, s)
+#define KVS_DM(GG, BB)                                                                               \
+    return launch_g<GG, BB>(q, kc, vc, bt, nt, B, Hq, Hkv, bs, max_blocks, scale_log2, tps, max_splits, \
+                            o, partials, status, s)
+#define KVS_DM_BS(GG)              \
+    if (bs == kDmChunk) KVS_DM(GG, kDmChunk); \
+    if (bs == 1) KVS_DM(GG, 1);    \
+    KVS_DM(GG, 0)
     switch (G) {
-        case 1: KVS_DM(1);
-        case 2: KVS_DM(2);
-        case 4: KVS_DM(4);
-        default: KVS_DM(8);
+        case 1: KVS_DM_BS(1);
+        case 2: KVS_DM_BS(2);
+        case 4: KVS_DM_BS(4);
+        default: KVS_DM_BS(8);
     }
+#undef KVS_DM_BS
 #undef KVS_DM
 }
 
