@@ -172,3 +172,23 @@ def test_decode_negative_block_id_reports():
     kvs.kvs_paged_decode_attn(torch.zeros((1, 1, d), dtype=torch.bfloat16, device="cuda"), kc, kc, bt,
                               dev(np.array([40], np.int32)), bs, 0.1, status=status)
     assert status.item() == kvs.KVS_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("bs", [4, 8, 32])
+def test_decode_other_block_sizes(bs):
+    """Block sizes other than 16 and 1 take the kernel's general addressing path
+    (the two the workloads use have their own); several splits per sequence."""
+    rng = np.random.default_rng(100 + bs)
+    B, Hkv, G, d = 3, 2, 4, 128
+    Hq = G * Hkv
+    M = (1600 + bs - 1) // bs
+    pool = B * M + 7
+    kc = W.round_bf16(rng.standard_normal((pool, Hkv, bs, d)).astype(np.float32))
+    vc = W.round_bf16(rng.standard_normal((pool, Hkv, bs, d)).astype(np.float32))
+    q = W.round_bf16(rng.standard_normal((B, Hq, d)).astype(np.float32))
+    bt = rng.permutation(pool)[: B * M].reshape(B, M).astype(np.int32)
+    nt = np.array([M * bs, M * bs - bs - 3, 5], np.int32)
+    o = host(kvs.kvs_paged_decode_attn(dev(q, torch.bfloat16), dev(kc, torch.bfloat16),
+                                       dev(vc, torch.bfloat16), dev(bt), dev(nt), bs, 1 / np.sqrt(d)))
+    want = oracle.paged_decode(q, kc, vc, bt, nt, bs, 1 / np.sqrt(d))
+    assert_close(o, want, BF16_TOL, f"decode bs={bs}")
