@@ -8,18 +8,19 @@
 //   dQ = scale dS K, dK = scale dS^T Q, D = rowsum(dO * O).
 //
 // Three launches, no atomics (deterministic):
-//   prep   D and LSE*log2(e) per (trace, head, row), padded to whole tiles
+//   prep   D and -LSE*log2(e) per (trace, head, row), padded to whole tiles
 //   dK/dV  one CTA per (key tile, kv head, trace); walks the column lists of
-//          the mask for every query head of the group. Transposed products
-//          S^T = K Q^T and dP^T = V dO^T put one key per TMEM lane, so P^T and
-//          dS^T are written back to TMEM in bf16 and used as the A operand of
-//          dV += P^T dO and dK += dS^T Q. Within a tile a key's visible query
-//          rows form one interval (j <= t < kappa_j), so masking needs only
-//          kappa_j, not the bit rows.
+//          the mask for every query head of the group, in items of 64 query
+//          rows. Transposed products S^T = K Q^T and dP^T = V dO^T put one key
+//          per TMEM lane, so P^T and dS^T are written back to TMEM in bf16 and
+//          used as the A operand of dV += P^T dO and dK += dS^T Q. Two TMEM
+//          buffers and two groups of elementwise warps take the items in turn.
+//          Within a tile a key's visible query rows form one interval
+//          (j <= t < kappa_j), so masking needs only kappa_j, not the bit rows.
 //   dQ     one CTA per (query tile, head, trace) over the row lists:
 //          S = Q K^T, dP = dO V^T, dS (bit-masked) to TMEM, dQ += dS K.
-// Warp roles as in the forward: warp 0 TMA, warp 1 TMEM + MMA issue, warps
-// 2..5 elementwise (thread = TMEM lane).
+// Warp roles: warp 0 TMA, warp 1 TMEM + MMA issue (the whole warp runs the
+// loop, one elected lane issues), warps 2..9 elementwise (thread = TMEM lane).
 #include "common.cuh"
 
 namespace kvs {

@@ -8,7 +8,8 @@
 //
 // One CTA per (query tile, head, trace), 6 warps:
 //   warp 0      TMA producer: Q once, then K and V tiles (2-stage rings each)
-//   warp 1      TMEM allocator and single-thread tcgen05.mma issuer
+//   warp 1      TMEM allocator and tcgen05.mma issue (the whole warp runs the
+//               loop, one lane chosen by elect.sync issues)
 //   warps 2..5  softmax: thread = TMEM lane = query row
 // TMEM (512 columns): S double buffer [0,128) [128,256), O accumulator [256,384).
 // Per tile n: S_n = Q K_n^T (SS MMA) -> softmax reads S_n, writes P_n as bf16
