@@ -370,6 +370,19 @@ def _src_hash(files):
     return h.hexdigest()[:12]
 
 
+def over_ranks(elapsed_ms: float, pairs: float, device):
+    """Job-wide figures of a timed region: the slowest rank's time and the visible
+    pairs of all ranks' traces. One collective of each kind, taken by every rank in
+    the same order; a single process returns its own figures."""
+    if not (torch.distributed.is_available() and torch.distributed.is_initialized()):
+        return elapsed_ms, pairs
+    t = torch.tensor([elapsed_ms], device=device, dtype=torch.float64)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    p = torch.tensor([pairs], device=device, dtype=torch.float64)
+    torch.distributed.all_reduce(p)
+    return float(t.item()), float(p.item())
+
+
 def run_ours(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -401,15 +414,7 @@ def run_ours(args):
     torch.cuda.synchronize()
     elapsed = t0.elapsed_time(t1)
     clk = clocks.stop() if clocks else None
-    if world > 1:
-        t = torch.tensor([elapsed], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        elapsed = float(t.item())
-        p = torch.tensor([float(step.pairs)], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(p)
-        pairs_all = float(p.item())
-    else:
-        pairs_all = float(step.pairs)
+    elapsed, pairs_all = over_ranks(elapsed, float(step.pairs), dev)
     assert step.status.item() == 0, f"device status {step.status.item()}"
     ms = elapsed / args.steps
     flops_step = FLOPS_PER_PAIR_D * cfg.d * pairs_all * cfg.hq
