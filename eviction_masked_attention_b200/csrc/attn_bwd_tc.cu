@@ -86,9 +86,6 @@ __device__ __forceinline__ void store_row64(__nv_bfloat16 *dst, const uint32_t (
     }
 }
 
-// TMEM column of the packed bf16 A operand for K-step kk when each half of the
-// 128 K values was packed at the start of its own 64-column region.
-__device__ __forceinline__ uint32_t packed_col(int kk) { return (kk < 4) ? kk * 8 : 64 + (kk - 4) * 8; }
 
 // ---------------------------------------------------------------------- dK / dV
 //

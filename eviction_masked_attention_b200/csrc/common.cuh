@@ -43,23 +43,6 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
-// 2^x evaluated on the FMA pipe, freeing the special-function unit (which also
-// executes conversions, so none are used): t = x + 1.5*2^23 rounds x to the
-// integer n held in the low mantissa bits of t; f = x - n lies in [-1/2, 1/2];
-// 2^f comes from a cubic fitted for minimum relative error on that interval
-// (eviction_masked_attention_b200/fit_exp2_poly.py; max relative error 1.5e-4 in
-// fp32, far below the 2^-9 of the bf16 P it feeds); n is added to the exponent
-// field by one integer multiply-add (bits(t) * 2^23 wraps to n * 2^23).
-// Arguments below -127 are clamped (result ~1e-38); valid up to x < 128.
-__device__ __forceinline__ float exp2_fma(float x) {
-    x = fmaxf(x, -127.f);
-    const float t = x + 12582912.f;
-    const float f = x - (t - 12582912.f);
-    const float p = fmaf(fmaf(fmaf(5.517166907e-02f, f, 2.426111222e-01f), f, 6.932609855e-01f), f,
-                         9.999280735e-01f);
-    return __uint_as_float(__float_as_uint(t) * 8388608u + __float_as_uint(p));
-}
-
 // Pairs of fp32 lanes in one 64-bit register, for the sm_100 f32x2 instructions
 // (one issue slot for two IEEE-rounded operations).
 __device__ __forceinline__ uint64_t f2_make(float a, float b) {
@@ -91,8 +74,15 @@ __device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
     return d;
 }
 
-// exp2_fma on two lanes with f32x2 arithmetic: the same operations, rounded the
-// same way per lane, in about half the issue slots.
+// 2^x for two lanes evaluated on the FMA pipe in f32x2 arithmetic, freeing the
+// special-function unit (which also executes conversions, so none are used):
+// t = x + 1.5*2^23 rounds x to the integer n held in the low mantissa bits of t;
+// f = x - n lies in [-1/2, 1/2]; 2^f comes from a cubic fitted for minimum
+// relative error on that interval (eviction_masked_attention_b200/fit_exp2_poly.py;
+// max relative error 1.5e-4 in fp32, far below the 2^-9 of the bf16 P it feeds);
+// n is added to the exponent field by one integer multiply-add (bits(t) * 2^23
+// wraps to n * 2^23). Arguments below -127 are clamped (result ~1e-38); valid up
+// to x < 128. Each lane is rounded exactly as the scalar sequence would be.
 __device__ __forceinline__ void exp2_fma_x2(float x0, float x1, float &y0, float &y1) {
     const uint64_t x = f2_make(fmaxf(x0, -127.f), fmaxf(x1, -127.f));
     const uint64_t magic = f2_make(12582912.f, 12582912.f);

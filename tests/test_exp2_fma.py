@@ -14,11 +14,13 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
 def _kernel_coeffs():
+    """(c0, c1, c2, c3) as written in exp2_fma_x2, where each appears once per lane."""
     src = open(os.path.join(ROOT, "eviction_masked_attention_b200", "csrc", "common.cuh")).read()
-    body = src[src.index("float exp2_fma("):]
-    body = body[body.index("const float p"): body.index("return")]
+    body = src[src.index("void exp2_fma_x2("):]
+    body = body[: body.index("f2_split(t")]
     vals = [float(v) for v in re.findall(r"([0-9]\.[0-9]+e[+-][0-9]+)f", body)]
-    c3, c2, c1, c0 = vals[:4]
+    assert len(vals) == 8 and vals[1::2] == vals[0::2]   # the same constant in both lanes
+    c3, c2, c1, c0 = vals[0::2]
     return np.array([c0, c1, c2, c3])
 
 
@@ -41,13 +43,3 @@ def test_relative_error_over_kernel_range():
     # exact powers of two stay within the same bound
     assert abs(_eval_fp32(c, np.array([0.0]))[0] - 1.0) < 2e-4
 
-
-def test_two_lane_variant_uses_the_same_constants():
-    src = open(os.path.join(ROOT, "eviction_masked_attention_b200", "csrc", "common.cuh")).read()
-    body = src[src.index("void exp2_fma_x2("):]
-    body = body[: body.index("f2_split(t")]
-    vals = [float(v) for v in re.findall(r"([0-9]\.[0-9]+e[+-][0-9]+)f", body)]
-    # each constant appears twice (one per lane), highest power first
-    c3, c2, c1, c0 = vals[0], vals[2], vals[4], vals[6]
-    assert vals[1::2] == vals[0::2]
-    np.testing.assert_array_equal(np.array([c0, c1, c2, c3]), _kernel_coeffs())
