@@ -182,7 +182,10 @@ kvs_status kvs_rope_logical(const void *x, int64_t x_tok_stride, void *y, const 
  *   block_table int32 [B][max_blocks]; num_tokens int32 [B] (0 gives o = 0)
  *   dt      KVS_BF16 with d = 128, or KVS_F32 with d = 64 (fp32 accumulation)
  *   ws      device scratch of kvs_paged_decode_ws_bytes(...) bytes (per-split
- *           partial results; no initialisation needed). The call runs one
+ *           partial results, B * Hq * splits * (d + 2) fp32; no initialisation
+ *           needed). A split covers 1024, 512, 256 or 128 entries: the largest
+ *           that still gives 148 CTAs when the sequences are half full; with a
+ *           single split the scratch is not used (16 bytes). The call runs one
  *           split kernel and, when a sequence spans several splits, a merge
  *           kernel.
  * A block id < 0 sets KVS_ERR_INVALID_ARG and its entries are skipped.

@@ -65,3 +65,25 @@ def test_product_path_has_no_oracle_import():
                 txt = open(os.path.join(dp, f)).read()
                 assert "import oracle" not in txt and "from oracle" not in txt, f
                 assert "oracle.c" not in txt, f
+
+
+def _plan_ws(B, Hq, Hkv, d, bs, max_blocks):
+    """The split plan as documented at kvs_paged_decode_ws_bytes: entries per split
+    tps in {1024, 512, 256, 128}, the largest that still gives 148 CTAs when the
+    sequences are half full; partials (d + 2 floats) per (sequence, query head, split)
+    only when a sequence can need more than one split."""
+    max_tok = max_blocks * bs
+    units = B * Hkv
+    tps = 1024
+    while tps > 128 and units * -(-(max_tok // 2) // tps) < 148:
+        tps //= 2
+    splits = max(1, -(-max_tok // tps))
+    return B * Hq * splits * (d + 2) * 4 if splits > 1 else 16
+
+
+@pytest.mark.parametrize("shape", [(64, 32, 8, 128, 16, 2049),   # paged workload
+                                   (2, 64, 8, 128, 1, 28701),    # two long sequences, 1-token blocks
+                                   (3, 8, 2, 128, 16, 100),      # few units: short splits
+                                   (1, 8, 1, 128, 16, 4)])       # one split: no partials
+def test_decode_plan_workspace(built, shape):
+    assert kvs.lib().kvs_paged_decode_ws_bytes(*shape) == _plan_ws(*shape)
