@@ -72,3 +72,11 @@ def test_ranks_take_distinct_traces():
     tail = both[both[:, 0] >= cfg.batch].copy()
     tail[:, 0] -= cfg.batch
     np.testing.assert_array_equal(e1, tail)
+
+
+def test_cpu_baseline_entry_extrapolates_linearly():
+    import bench
+
+    e = bench.cpu_baseline_entry(2.0e12, 4.0, 16, 1.0e15, "sample")
+    assert e["value"] == 0.5 and e["unit"] == "TFLOP/s" and e["kind"] == "oracle" and e["cores"] == 16
+    assert e["extrapolated_full_step_s"] == 2000.0
