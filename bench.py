@@ -455,9 +455,9 @@ def run_ours(args):
         dec_gbs = dec_b / (dur["decode"] * 1e-3) / 1e9
         cpu = None
         if not args.no_cpu_baseline and world == 1:
-            f, s, thr = oracle_sample(cfg, 3072)
+            f, s, thr = oracle_sample(cfg, 2560)
             cpu = cpu_baseline_entry(f, s, thr, flops_step,
-                                     "first 3072 tokens of trace 0, one kv group (8 query heads), "
+                                     "first 2560 tokens of trace 0, one kv group (8 query heads), "
                                      f"fwd + full bwd, {s:.1f} s")
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
