@@ -211,6 +211,20 @@ def dkdv_cols(qg, k, v, dog, kap_b, scale: float, cols):
     return dk, dv
 
 
+def dkdv_cols_fwd(qg, k, v, dog, og, lseg, kap_b, scale: float, cols):
+    """dK, dV for key positions ``cols`` of one group from the forward's per-row
+    O and LSE (qg/dog/og [G,N,d], lseg [G,N], k/v [N,d]). Rows with dO = 0 add
+    nothing; their og/lseg may be 0/+inf."""
+    qg, dog, og, lseg, k, v = _f64(qg), _f64(dog), _f64(og), _f64(lseg), _f64(k), _f64(v)
+    cs, kb = _i32(cols), _i32(kap_b)
+    G, N, d = qg.shape
+    dk, dv = np.empty((len(cs), d)), np.empty((len(cs), d))
+    _L().orc_attn_dkdv_cols_fwd(_p(qg), _p(k), _p(v), _p(dog), _p(og), _p(lseg), _p(kb),
+                                C.c_int32(N), C.c_int32(G), C.c_int32(d), C.c_double(scale),
+                                _p(cs), C.c_int64(len(cs)), _p(dk), _p(dv))
+    return dk, dv
+
+
 # ------------------------------------------------------------------ paged cache
 
 def compact(block_table, block_lpos, num_blocks, num_tokens, block_size: int, events):
@@ -241,11 +255,32 @@ def paged_decode(q, k_cache, v_cache, block_table, num_tokens, block_size: int, 
 
 # ------------------------------------------------------------------ toy model
 
+def toy_project(x, W) -> np.ndarray:
+    """The toy model's projection, row by row: y[n] = x[n] W (x [n, Din], W [Din, Dout])."""
+    x, W = _f64(x), _f64(W)
+    n, Din = x.shape
+    Dout = W.shape[1]
+    y = np.empty((n, Dout))
+    _L().orc_toy_project(_p(x), _p(W), C.c_int64(n), C.c_int32(Din), C.c_int32(Dout), _p(y))
+    return y
+
+
+def toy_rotate(x, lpos, theta: float) -> np.ndarray:
+    """The toy model's rotation of x [n, H, d] at positions lpos[n] (returns a copy)."""
+    y = _f64(x).copy()
+    n, H, d = y.shape
+    assert d % 2 == 0 and d <= 512
+    _L().orc_toy_rotate(_p(y), _p(_i32(lpos)), C.c_int64(n), C.c_int32(H), C.c_int32(d),
+                        C.c_double(theta))
+    return y
+
+
 class Toy:
     """Random-weight L-layer attention stack used to check that the replay
     reproduces generation with physical eviction at every layer."""
 
     def __init__(self, L, Dm, Hq, Hkv, d, theta, seed):
+        assert d % 2 == 0 and d <= 512 and Hq % Hkv == 0
         rng = np.random.default_rng(seed)
         self.L, self.Dm, self.Hq, self.Hkv, self.d, self.theta = L, Dm, Hq, Hkv, d, theta
         self.scale = 1.0 / np.sqrt(d)

@@ -14,14 +14,14 @@
  *    found through a block table, and compaction removes whole blocks and joins
  *    the remaining references with no holes; the SGLang setup uses 1-token
  *    blocks; every compaction event is recorded during generation and the
- *    trainer replays the continuous trace with later tokens blocked from spans
- *    inference had already removed.
+ *    trainer replays the continuous trace, masking from each query the spans
+ *    that an eviction at or before its position had removed.
  *  - "KV-streams for Efficient Compaction in Agentic Reinforcement Learning"
  *    (paper listing), Fig. 2(A): re-prefill recomputes the retained tokens,
  *    KV-streams trains on one continuous trace with an attention mask that
  *    reproduces eviction.
  *
- * Readings where the pages are silent (each also listed in the design notes):
+ * Readings where the pages are silent:
  *  - an event (seq, tau, start, end) removes logical positions [start, end)
  *    before the token at logical position tau is generated; so key j is
  *    visible to query t iff j <= t < kappa_j, kappa_j = min tau over the
@@ -185,24 +185,25 @@ int orc_tile_lists(const int32_t *kappa, const uint8_t *cls, int32_t B, int32_t 
 /* ------------------------------------------------------------------------- */
 
 /* y[n][h][:] = R(+-lpos[n]) x[n][h][:], rotate-half pairs (i, i + d/2). */
+/* One head row of d values rotated by the angle of position p (rotate-half). */
+static void rope_row(const double *xr, double *yr, int32_t d, double p, double theta) {
+    const int32_t half = d / 2;
+    for (int32_t i = 0; i < half; ++i) {
+        double ang = p * pow(theta, -2.0 * (double)i / (double)d);
+        double c = cos(ang), s = sin(ang);
+        double a = xr[i], b = xr[i + half];
+        yr[i] = a * c - b * s;
+        yr[i + half] = a * s + b * c;
+    }
+}
+
 void orc_rope(const double *x, double *y, const int32_t *lpos, int64_t n_tok, int32_t H,
               int32_t d, double theta, int32_t inverse) {
-    const int32_t half = d / 2;
 #pragma omp parallel for schedule(static)
     for (int64_t n = 0; n < n_tok; ++n) {
         double p = (double)lpos[n];
         if (inverse) p = -p;
-        for (int32_t h = 0; h < H; ++h) {
-            const double *xr = x + (n * H + h) * d;
-            double *yr = y + (n * H + h) * d;
-            for (int32_t i = 0; i < half; ++i) {
-                double ang = p * pow(theta, -2.0 * (double)i / (double)d);
-                double c = cos(ang), s = sin(ang);
-                double a = xr[i], b = xr[i + half];
-                yr[i] = a * c - b * s;
-                yr[i + half] = a * s + b * c;
-            }
-        }
+        for (int32_t h = 0; h < H; ++h) rope_row(x + (n * H + h) * d, y + (n * H + h) * d, d, p, theta);
     }
 }
 
@@ -418,6 +419,45 @@ void orc_attn_dkdv_cols(const double *q, const double *k, const double *v, const
     }
 }
 
+/*
+ * dK, dV for key positions cols[r] of a group of G query heads, given each
+ * query row's forward output o[g][t] and log-sum-exp lse[g][t] (as returned by
+ * orc_attn_rows): the textbook formulas summed over the rows that see j,
+ *   P_tj = exp(scale <q_t,k_j> - LSE_t),  D_t = <dO_t, O_t>,
+ *   dV_j = sum_{g,t} P_tj dO_t,  dK_j = scale sum_{g,t} P_tj (<dO_t,v_j> - D_t) q_t.
+ * A row whose dO is zero contributes nothing; callers may pass o = 0 and
+ * lse = +inf for such rows (then P_tj = 0).
+ */
+void orc_attn_dkdv_cols_fwd(const double *q, const double *k, const double *v,
+                            const double *dout, const double *o, const double *lse,
+                            const int32_t *kappa, int32_t N, int32_t G, int32_t d, double scale,
+                            const int32_t *cols, int64_t ncol, double *dk, double *dv) {
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t r = 0; r < ncol; ++r) {
+        int64_t j = cols[r];
+        double *dkj = dk + r * d, *dvj = dv + r * d;
+        for (int32_t i = 0; i < d; ++i) dkj[i] = dvj[i] = 0.0;
+        for (int32_t g = 0; g < G; ++g) {
+            for (int64_t t = j; t < N; ++t) {
+                if (!orc_visible(kappa, N, t, j)) continue;
+                const double *qt = q + ((int64_t)g * N + t) * d;
+                const double *dot = dout + ((int64_t)g * N + t) * d;
+                const double *ot = o + ((int64_t)g * N + t) * d;
+                double D = 0.0, s = 0.0, dp = 0.0;
+                for (int32_t i = 0; i < d; ++i) D += dot[i] * ot[i];
+                for (int32_t i = 0; i < d; ++i) s += qt[i] * k[j * d + i];
+                for (int32_t i = 0; i < d; ++i) dp += dot[i] * v[j * d + i];
+                double P = exp(scale * s - lse[(int64_t)g * N + t]);
+                double dS = P * (dp - D);
+                for (int32_t i = 0; i < d; ++i) {
+                    dvj[i] += P * dot[i];
+                    dkj[i] += scale * dS * qt[i];
+                }
+            }
+        }
+    }
+}
+
 /* ------------------------------------------------------------------------- */
 /* Paged cache: block-table compaction and decode                            */
 /* ------------------------------------------------------------------------- */
@@ -518,18 +558,27 @@ static void toy_proj(const double *x, const double *W, int32_t Din, int32_t Dout
         for (int32_t c = 0; c < Dout; ++c) y[c] += x[r] * W[(int64_t)r * Dout + c];
 }
 
+/* Rotate the H head rows of x in place at logical position pos: the same
+ * per-row rotation as orc_rope. */
 static void toy_rotate(double *x, int32_t H, int32_t d, double pos, double theta) {
-    const int32_t half = d / 2;
+    double tmp[512];
     for (int32_t h = 0; h < H; ++h) {
         double *r = x + (int64_t)h * d;
-        for (int32_t i = 0; i < half; ++i) {
-            double ang = pos * pow(theta, -2.0 * (double)i / (double)d);
-            double c = cos(ang), s = sin(ang);
-            double a = r[i], b = r[i + half];
-            r[i] = a * c - b * s;
-            r[i + half] = a * s + b * c;
-        }
+        rope_row(r, tmp, d, pos, theta);
+        memcpy(r, tmp, sizeof(double) * (size_t)d);
     }
+}
+
+/* Test hooks for the toy model's two building blocks: y[n] = x[n] W for n rows
+ * (toy_proj), and the in-place rotation of n tokens of H heads (toy_rotate). */
+void orc_toy_project(const double *x, const double *W, int64_t n, int32_t Din, int32_t Dout,
+                     double *y) {
+    for (int64_t r = 0; r < n; ++r) toy_proj(x + r * Din, W, Din, Dout, y + r * Dout);
+}
+
+void orc_toy_rotate(double *x, const int32_t *lpos, int64_t n, int32_t H, int32_t d,
+                    double theta) {
+    for (int64_t r = 0; r < n; ++r) toy_rotate(x + r * H * d, H, d, (double)lpos[r], theta);
 }
 
 /* A per-layer paged cache: pool of blocks, free list, block table. */

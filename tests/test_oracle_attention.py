@@ -133,6 +133,48 @@ def test_sampled_rows_and_cols_agree_with_full_bwd():
         np.testing.assert_allclose(gv, dv[0, cols, kvh], atol=1e-12, rtol=0)
 
 
+def _autograd_dkdv(q, k, v, do, ev, b, scale):
+    """dK, dV of one trace from torch autograd through fp64 SDPA with the event-wise mask."""
+    N = q.shape[1]
+    mask = torch.from_numpy(dense_mask_eventwise(ev, b, N))
+    qt = torch.from_numpy(np.transpose(q[b], (1, 0, 2))).requires_grad_(True)
+    kt = torch.from_numpy(np.transpose(k[b], (1, 0, 2))).requires_grad_(True)
+    vt = torch.from_numpy(np.transpose(v[b], (1, 0, 2))).requires_grad_(True)
+    out = _sdpa(qt, kt, vt, mask, scale)
+    out.backward(torch.from_numpy(np.transpose(do[b], (1, 0, 2))))
+    return kt.grad.numpy(), vt.grad.numpy()
+
+
+@pytest.mark.parametrize("banded", [False, True])
+def test_dkdv_cols_from_forward_rows(banded):
+    """dK/dV by column from the forward's per-row O and LSE equals autograd; with dO
+    zero outside a few row bands, rows outside them may carry O = 0, LSE = +inf."""
+    ev, q, k, v, do = _case(7, N=260, Hq=6, Hkv=2, d=16, B=1)
+    N, Hq, d = q.shape[1], q.shape[2], q.shape[3]
+    Hkv = k.shape[2]
+    G = Hq // Hkv
+    scale = 1 / np.sqrt(d)
+    rows = np.arange(N)
+    if banded:
+        band = ((rows >= 40) & (rows < 70)) | (rows >= 230)
+        do = do * band[None, :, None, None]
+    kap = oracle.kappa(ev, 1, N)
+    gk_all, gv_all = _autograd_dkdv(q, k, v, do, ev, 0, scale)
+    cols = np.array([0, 1, 39, 41, 100, 200, 259])
+    for kvh in range(Hkv):
+        hs = slice(kvh * G, (kvh + 1) * G)
+        qg = np.transpose(q[0, :, hs], (1, 0, 2)); dog = np.transpose(do[0, :, hs], (1, 0, 2))
+        og, lg = np.empty((G, N, d)), np.empty((G, N))
+        for g in range(G):
+            og[g], lg[g] = oracle.attn_rows(qg[g], rows, k[0, :, kvh], v[0, :, kvh], kap[0], scale)
+        if banded:
+            og[:, ~band] = 0.0
+            lg[:, ~band] = np.inf
+        gk, gv = oracle.dkdv_cols_fwd(qg, k[0, :, kvh], v[0, :, kvh], dog, og, lg, kap[0], scale, cols)
+        np.testing.assert_allclose(gk, gk_all[kvh, cols], atol=1e-11, rtol=0)
+        np.testing.assert_allclose(gv, gv_all[kvh, cols], atol=1e-11, rtol=0)
+
+
 def test_dk_sums_to_zero_per_group():
     # sum_j dS_tj = 0 for every query row, so sum_j dK_j = 0 (a property at any size)
     ev, q, k, v, do = _case(9, N=160)

@@ -56,3 +56,60 @@ def test_reprefill_differs_after_first_event():
     assert diff.min() > 1e-3                                 # every later token differs
     # layer-2 attention (built on layer-1 states the evicted span influenced) differs too
     assert np.abs(a_s[t0:, 1] - a_p[t0:, 1]).max() > 1e-2
+
+
+# ------------------------------------------------------------------ the toy model's parts
+#
+# Generation and replay above share the toy's projection and rotation, so the
+# bit-identity pin cannot see a mistake in either. These pin them separately:
+# the projection against numpy's matrix product, the rotation against the
+# pinned rotary oracle and its invariants, and one whole layer against a
+# composition of pinned pieces.
+
+def test_toy_projection_is_a_matrix_product():
+    rng = np.random.default_rng(0)
+    for n, din, dout in ((1, 3, 5), (7, 24, 32), (4, 16, 8)):
+        x, w = rng.standard_normal((n, din)), rng.standard_normal((din, dout))
+        np.testing.assert_allclose(oracle.toy_project(x, w), np.matmul(x, w), rtol=1e-13, atol=1e-13)
+
+
+@pytest.mark.parametrize("H,d,theta", [(1, 8, 1e4), (4, 8, 1e4), (3, 64, 5e5)])
+def test_toy_rotation_is_the_rotary_embedding(H, d, theta):
+    rng = np.random.default_rng(H * d)
+    n = 9
+    x = rng.standard_normal((n, H, d))
+    lp = rng.integers(0, 131072, n).astype(np.int32)
+    y = oracle.toy_rotate(x, lp, theta)
+    np.testing.assert_allclose(y, oracle.rope(x, lp, theta), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(np.linalg.norm(y, axis=-1), np.linalg.norm(x, axis=-1), rtol=1e-12)
+    # rotary dot products depend on the position difference only, head by head
+    c = 777
+    y2 = oracle.toy_rotate(x, lp + c, theta)
+    d1 = np.einsum("hd,hd->h", y[0], y[1])
+    d2 = np.einsum("hd,hd->h", y2[0], y2[1])
+    np.testing.assert_allclose(d1, d2, rtol=1e-9, atol=1e-9)
+    # a row is rotated with its own position: rotating row 1 alone at its position agrees
+    np.testing.assert_allclose(oracle.toy_rotate(x[1:2], lp[1:2], theta), y[1:2], rtol=0, atol=0)
+
+
+@pytest.mark.parametrize("with_events", [False, True])
+def test_toy_layer_is_projection_rotation_masked_attention(with_events):
+    """One toy layer = numpy projections -> pinned rotation -> pinned masked attention
+    forward -> numpy output projection added to the residual."""
+    N, Dm, Hq, Hkv, d, theta = 96, 12, 4, 2, 8, 1e4
+    toy = oracle.Toy(L=1, Dm=Dm, Hq=Hq, Hkv=Hkv, d=d, theta=theta, seed=3)
+    x0 = np.random.default_rng(4).standard_normal((N, Dm))
+    ev = np.array([[0, 40, 8, 24], [0, 70, 24, 40]], np.int32) if with_events else np.zeros((0, 4), np.int32)
+    kap = oracle.kappa(ev, 1, N)
+    xr, ar = toy.replay(x0, kap[0])
+    lp = np.arange(N, dtype=np.int32)
+    q = oracle.rope((x0 @ toy.Wq[0]).reshape(N, Hq, d), lp, theta)
+    k = oracle.rope((x0 @ toy.Wk[0]).reshape(N, Hkv, d), lp, theta)
+    v = (x0 @ toy.Wv[0]).reshape(N, Hkv, d)
+    o, _ = oracle.attn_fwd(q[None], k[None], v[None], kap, toy.scale)
+    a = o[0].reshape(N, Hq * d)
+    np.testing.assert_allclose(ar[:, 0], a, rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(xr, x0 + a @ toy.Wo[0], rtol=1e-10, atol=1e-12)
+    if with_events:
+        _, xg, ag, *_ = toy.generate(x0, ev[:, 1:4], 8, pool=N // 8 + 4)
+        np.testing.assert_allclose(ag[:, 0], a, rtol=1e-10, atol=1e-12)
