@@ -73,12 +73,14 @@ def lib() -> C.CDLL:
         L.kvs_build_tile_mask.argtypes = [vp, i32, i32, i32, C.POINTER(_TileMaskC), C.POINTER(_SizesC),
                                           vp, sz, vp]
         L.kvs_compact_block_table.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, vp, i32, vp, vp, vp, vp]
-        L.kvs_rope_logical.argtypes = [vp, i64, vp, vp, i32, i32, i32, f64, i32, vp, i32, vp, i64, vp,
-                                       i32, vp, vp]
+        L.kvs_rope_logical.argtypes = [vp, i64, vp, vp, i32, i32, i32, f64, i32, vp, i32, i32, vp, i64,
+                                       vp, i32, vp, vp]
         L.kvs_paged_decode_ws_bytes.argtypes = [i32, i32, i32, i32, i32, i32]
         L.kvs_paged_decode_ws_bytes.restype = sz
-        L.kvs_paged_decode_attn.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, i32,
-                                            vp, vp, sz, vp, vp]
+        L.kvs_paged_decode_attn.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, f32,
+                                            i32, vp, vp, sz, vp, vp]
+        L.kvs_paged_decode_attn_static.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32,
+                                                   f32, i32, vp, vp, vp]
         L.kvs_masked_attn_fwd.argtypes = [vp, vp, vp, C.POINTER(_TileMaskC), i32, i32, i32, i32, i32,
                                           f32, i32, vp, vp, vp, vp, vp]
         L.kvs_masked_attn_bwd_ws_bytes.argtypes = [i32, i32, i32, i32, i32, i32]
@@ -90,7 +92,8 @@ def lib() -> C.CDLL:
         L.kvs_version.restype = i32
         L.kvs_last_cuda_error.restype = C.c_char_p
         for r in ("kvs_build_tile_mask", "kvs_compact_block_table", "kvs_rope_logical",
-                  "kvs_paged_decode_attn", "kvs_masked_attn_fwd", "kvs_masked_attn_bwd"):
+                  "kvs_paged_decode_attn", "kvs_paged_decode_attn_static", "kvs_masked_attn_fwd",
+                  "kvs_masked_attn_bwd"):
             getattr(L, r).restype = i32
         _lib = L
     return _lib
@@ -222,7 +225,8 @@ def kvs_rope_logical(x, lpos, theta: float, inverse: bool = False, out=None, out
                      block_size: int = 1, v=None, v_out=None, status=None):
     """Rotate x[n, H, d] (or a row-strided 2-D view [n, stride] holding H*d) at logical
     positions lpos[n]. With out_slot, write rotated rows into the paged cache ``out``
-    [pool, H, bs, d] and copy v rows into ``v_out`` at the same slots."""
+    [pool, H, bs, d] and copy v rows into ``v_out`` at the same slots; the cache's
+    first dimension is passed as the pool size the slots are checked against."""
     n = lpos.numel()
     H, d = x.shape[-2], x.shape[-1]
     if x.stride(-1) != 1 or x.stride(-2) != d:
@@ -234,8 +238,9 @@ def kvs_rope_logical(x, lpos, theta: float, inverse: bool = False, out=None, out
     if status is None:
         status = torch.zeros(1, dtype=torch.int32, device=x.device)
     vs = v.stride(0) if v is not None else 0
+    pool = out.shape[0] if out_slot is not None else 0
     _check(lib().kvs_rope_logical(_p(x), x.stride(0), _p(out), _p(lpos), n, H, d, float(theta),
-                                  int(inverse), _p(out_slot), block_size, _p(v), vs, _p(v_out),
+                                  int(inverse), _p(out_slot), block_size, pool, _p(v), vs, _p(v_out),
                                   _dtype_code(x), _p(status), _stream()), "kvs_rope_logical")
     return out
 
@@ -244,7 +249,8 @@ def kvs_rope_logical(x, lpos, theta: float, inverse: bool = False, out=None, out
 
 def kvs_paged_decode_attn(q, k_cache, v_cache, block_table, num_tokens, block_size: int, scale: float,
                           out=None, ws=None, status=None):
-    """q [B, Hq, d]; caches [pool, Hkv, bs, d]; returns o [B, Hq, d]."""
+    """q [B, Hq, d]; caches [pool, Hkv, bs, d]; returns o [B, Hq, d]. Block ids are
+    checked against the caches' pool size."""
     _dev(q, k_cache, v_cache, block_table, num_tokens)
     B, Hq, d = q.shape
     Hkv = k_cache.shape[1]
@@ -258,8 +264,9 @@ def kvs_paged_decode_attn(q, k_cache, v_cache, block_table, num_tokens, block_si
     if status is None:
         status = torch.zeros(1, dtype=torch.int32, device=q.device)
     _check(L.kvs_paged_decode_attn(_p(q), _p(k_cache), _p(v_cache), _p(block_table), _p(num_tokens), B,
-                                   Hq, Hkv, d, block_size, M, float(scale), _dtype_code(q), _p(out),
-                                   _p(ws), ws.numel(), _p(status), _stream()), "kvs_paged_decode_attn")
+                                   Hq, Hkv, d, block_size, M, k_cache.shape[0], float(scale),
+                                   _dtype_code(q), _p(out), _p(ws), ws.numel(), _p(status), _stream()),
+           "kvs_paged_decode_attn")
     return out
 
 

@@ -39,8 +39,8 @@ template <typename T, int D>
 __global__ void k_rope(const T *__restrict__ x, int64_t x_stride, T *__restrict__ y,
                        const int32_t *__restrict__ lpos, int32_t n_tok, int32_t H, double log2_theta,
                        int32_t inverse, const int64_t *__restrict__ out_slot, int32_t bs,
-                       const T *__restrict__ v, int64_t v_stride, T *__restrict__ v_out,
-                       int32_t *status) {
+                       int64_t n_slots, const T *__restrict__ v, int64_t v_stride,
+                       T *__restrict__ v_out, int32_t *status) {
     constexpr int kThreadsPerHead = D / 8;  // each thread: 4 pairs
     const int32_t n = blockIdx.x;
     if (n >= n_tok) return;
@@ -61,8 +61,8 @@ __global__ void k_rope(const T *__restrict__ x, int64_t x_stride, T *__restrict_
     int64_t orow = 0;
     bool to_cache = out_slot != nullptr;
     if (to_cache) {
-        int64_t slot = out_slot[n];
-        if (slot < 0) {
+        const int64_t slot = out_slot[n];
+        if (slot < 0 || slot >= n_slots) {  // outside the cache: reported, row skipped
             if (threadIdx.x == 0) set_status(status, KVS_ERR_INVALID_ARG);
             return;
         }
@@ -100,9 +100,9 @@ using namespace kvs;
 extern "C" kvs_status kvs_rope_logical(const void *x, int64_t x_tok_stride, void *y,
                                        const int32_t *lpos, int32_t n_tok, int32_t H, int32_t d,
                                        double theta, int32_t inverse, const int64_t *out_slot,
-                                       int32_t block_size, const void *v, int64_t v_tok_stride,
-                                       void *v_out, kvs_dtype dt, int32_t *dev_status,
-                                       kvs_stream_t stream) {
+                                       int32_t block_size, int32_t pool_blocks, const void *v,
+                                       int64_t v_tok_stride, void *v_out, kvs_dtype dt,
+                                       int32_t *dev_status, kvs_stream_t stream) {
     if (n_tok < 0 || H <= 0 || !(theta > 1.0)) return KVS_ERR_INVALID_ARG;
     if (n_tok == 0) return KVS_OK;
     if (!x || !y || !lpos) return KVS_ERR_INVALID_ARG;
@@ -113,8 +113,10 @@ extern "C" kvs_status kvs_rope_logical(const void *x, int64_t x_tok_stride, void
     // vector accesses: 8 bytes (bf16) / 16 bytes (fp32) per thread
     const uintptr_t need = dt == KVS_F32 ? 16 : 8;
     if (((uintptr_t)x | (uintptr_t)y) % need || (x_tok_stride * esz) % need) return KVS_ERR_INVALID_ARG;
+    int64_t n_slots = 0;
     if (out_slot) {
-        if (block_size <= 0) return KVS_ERR_INVALID_ARG;
+        if (block_size <= 0 || pool_blocks <= 0) return KVS_ERR_INVALID_ARG;
+        n_slots = (int64_t)pool_blocks * block_size;
         if (v) {
             if (!v_out || v_tok_stride < (int64_t)H * d) return KVS_ERR_INVALID_ARG;
             if (((uintptr_t)v | (uintptr_t)v_out) % need || (v_tok_stride * esz) % need)
@@ -132,24 +134,24 @@ extern "C" kvs_status kvs_rope_logical(const void *x, int64_t x_tok_stride, void
         if (d == 64)
             k_rope<float, 64><<<n_tok, threads, 0, s>>>((const float *)x, x_tok_stride, (float *)y,
                                                         lpos, n_tok, H, l2t, inverse, out_slot,
-                                                        block_size, (const float *)v, v_tok_stride,
+                                                        block_size, n_slots, (const float *)v, v_tok_stride,
                                                         (float *)v_out, dev_status);
         else
             k_rope<float, 128><<<n_tok, threads, 0, s>>>((const float *)x, x_tok_stride, (float *)y,
                                                          lpos, n_tok, H, l2t, inverse, out_slot,
-                                                         block_size, (const float *)v, v_tok_stride,
+                                                         block_size, n_slots, (const float *)v, v_tok_stride,
                                                          (float *)v_out, dev_status);
     } else {
         using bf = __nv_bfloat16;
         if (d == 64)
             k_rope<bf, 64><<<n_tok, threads, 0, s>>>((const bf *)x, x_tok_stride, (bf *)y, lpos,
                                                      n_tok, H, l2t, inverse, out_slot, block_size,
-                                                     (const bf *)v, v_tok_stride, (bf *)v_out,
+                                                     n_slots, (const bf *)v, v_tok_stride, (bf *)v_out,
                                                      dev_status);
         else
             k_rope<bf, 128><<<n_tok, threads, 0, s>>>((const bf *)x, x_tok_stride, (bf *)y, lpos,
                                                       n_tok, H, l2t, inverse, out_slot, block_size,
-                                                      (const bf *)v, v_tok_stride, (bf *)v_out,
+                                                      n_slots, (const bf *)v, v_tok_stride, (bf *)v_out,
                                                       dev_status);
     }
     return cuda_status(cudaGetLastError());

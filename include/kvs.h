@@ -17,7 +17,10 @@
  *  - All tensor pointers are DEVICE pointers owned by the caller, unless a
  *    parameter says "host". The library allocates no memory and keeps no
  *    state between calls; scratch space is passed in as `ws` of the size the
- *    matching *_ws_bytes() query returns.
+ *    matching *_ws_bytes() query returns. The one exception is
+ *    kvs_paged_decode_attn_static: its scratch is a fixed 16 MiB array in the
+ *    library's device image, and it caches that array's device address per
+ *    device and CUDA context (see its comment).
  *  - Every call is asynchronous on `stream`, except kvs_build_tile_mask, which
  *    synchronises `stream` once to learn the sizes of its outputs.
  *  - Errors the host can see (NULL or misaligned pointers, bad sizes,
@@ -59,8 +62,9 @@ typedef enum {
 typedef enum { KVS_F32 = 0, KVS_BF16 = 1 } kvs_dtype;
 
 /* One compaction event: logical positions [start, end) of sequence `seq`
- * removed before the token at logical position `tau` ([T]: "records every
- * compaction event during generation"). Requires 0 <= start < end <= tau. */
+ * removed before the token at logical position `tau` is generated. Inference
+ * logs one such record per eviction and the trainer replays the log ([T],
+ * trainer replay). Requires 0 <= start < end <= tau. */
 typedef struct {
     int32_t seq, tau, start, end;
 } kvs_evict_range;
@@ -121,8 +125,9 @@ kvs_status kvs_build_tile_mask(const kvs_evict_range *ev, int32_t n_ev, int32_t 
                                kvs_stream_t stream);
 
 /*
- * Block-table compaction ([T] second fix: "removes complete blocks and joins
- * the remaining block references together"). In place, per sequence b:
+ * Block-table compaction ([T] second fix: only whole blocks leave the cache,
+ * and the surviving references are packed together so the table has no
+ * holes). In place, per sequence b:
  * every live entry i < num_blocks[b] whose logical span
  * [block_lpos[b][i], block_lpos[b][i] + block_size) lies inside one of the
  * sequence's ranges is removed; the others keep their order and move down;
@@ -155,19 +160,21 @@ kvs_status kvs_compact_block_table(int32_t *block_table, int32_t *block_lpos, in
  *   x       [n_tok] rows of H*d elements; row n starts at x + n*x_tok_stride
  *           (elements; heads contiguous within a row)
  *   lpos    int32 [n_tok]
- *   out_slot NULL: y is [n_tok][H][d] contiguous.
- *           non-NULL (int64 [n_tok]): y is a paged cache [pool][H][block_size][d]
- *           and row n goes to slot out_slot[n] (block slot/bs, offset slot%bs);
- *           then, if v != NULL, v rows (same stride rules, v_tok_stride) are
- *           copied unrotated to the same slots of v_out (the value cache).
- *           Slots must be >= 0 (a negative slot skips the row, sets
- *           KVS_ERR_INVALID_ARG).
+ *   out_slot NULL: y is [n_tok][H][d] contiguous (block_size and
+ *           pool_blocks are ignored).
+ *           non-NULL (int64 [n_tok]): y is a paged cache
+ *           [pool_blocks][H][block_size][d] and row n goes to slot out_slot[n]
+ *           (block slot/bs, offset slot%bs); then, if v != NULL, v rows (same
+ *           stride rules, v_tok_stride) are copied unrotated to the same slots
+ *           of v_out (the value cache, same shape). A slot outside
+ *           [0, pool_blocks * block_size) sets KVS_ERR_INVALID_ARG in
+ *           *dev_status and its row is skipped: nothing is written for it.
  *   dt      KVS_BF16 or KVS_F32 for x, y, v, v_out; d in {64, 128}.
  */
 kvs_status kvs_rope_logical(const void *x, int64_t x_tok_stride, void *y, const int32_t *lpos,
                             int32_t n_tok, int32_t H, int32_t d, double theta, int32_t inverse,
-                            const int64_t *out_slot, int32_t block_size, const void *v,
-                            int64_t v_tok_stride, void *v_out, kvs_dtype dt,
+                            const int64_t *out_slot, int32_t block_size, int32_t pool_blocks,
+                            const void *v, int64_t v_tok_stride, void *v_out, kvs_dtype dt,
                             int32_t *dev_status, kvs_stream_t stream);
 
 /*
@@ -178,25 +185,34 @@ kvs_status kvs_rope_logical(const void *x, int64_t x_tok_stride, void *y, const 
  * over live entries i < num_tokens[b]; entry i is offset i % block_size of
  * block block_table[b][i / block_size]. kv head = h / (Hq / Hkv).
  *   q, o     [B][Hq][d] (q already rotated at its logical position)
- *   k_cache, v_cache  [pool][Hkv][block_size][d]
+ *   k_cache, v_cache  [pool_blocks][Hkv][block_size][d]
  *   block_table int32 [B][max_blocks]; num_tokens int32 [B] (0 gives o = 0)
+ *   max_blocks * block_size must fit in int32 (else KVS_ERR_CAPACITY).
  *   dt      KVS_BF16 with d = 128, or KVS_F32 with d = 64 (fp32 accumulation)
- *   ws      device scratch of kvs_paged_decode_ws_bytes(...) bytes (per-split
- *           partial results, B * Hq * splits * (d + 2) fp32; no initialisation
- *           needed). A split covers 1024, 512, 256 or 128 entries: the largest
- *           that still gives 148 CTAs when the sequences are half full; with a
- *           single split the scratch is not used (16 bytes). The call runs one
- *           split kernel and, when a sequence spans several splits, a merge
- *           kernel.
- * A block id < 0 sets KVS_ERR_INVALID_ARG and its entries are skipped.
+ *   ws      device scratch of kvs_paged_decode_ws_bytes(...) bytes; no
+ *           initialisation needed. Work split: the live entries of unit
+ *           (b, kv head) are cut into chunks of 16; the units' chunks are laid
+ *           end to end and C CTAs take equal consecutive shares of them
+ *           (C = ceil(B*Hkv*ceil(max_blocks*block_size/16) / 72), rounded up to
+ *           a multiple of 444 = 148 SMs x 3, at most the chunk count), so the
+ *           split follows the actual num_tokens, found on the device. Scratch =
+ *           8*(B+1) bytes of prefix counts (rounded up to 256) + (C + B*Hkv)
+ *           partial results of G*(d+2) fp32. The call runs the split kernel
+ *           and a merge kernel.
+ * Errors found in device data set KVS_ERR_INVALID_ARG in *dev_status:
+ *  - a block id outside [0, pool_blocks): none of its entries is read; they
+ *    are left out of the softmax (as if evicted);
+ *  - num_tokens[b] < 0 or > max_blocks * block_size: the count is clamped to
+ *    that range.
  */
 size_t kvs_paged_decode_ws_bytes(int32_t B, int32_t Hq, int32_t Hkv, int32_t d, int32_t block_size,
                                  int32_t max_blocks);
 kvs_status kvs_paged_decode_attn(const void *q, const void *k_cache, const void *v_cache,
                                  const int32_t *block_table, const int32_t *num_tokens, int32_t B,
                                  int32_t Hq, int32_t Hkv, int32_t d, int32_t block_size,
-                                 int32_t max_blocks, float scale, kvs_dtype dt, void *o, void *ws,
-                                 size_t ws_bytes, int32_t *dev_status, kvs_stream_t stream);
+                                 int32_t max_blocks, int32_t pool_blocks, float scale,
+                                 kvs_dtype dt, void *o, void *ws, size_t ws_bytes,
+                                 int32_t *dev_status, kvs_stream_t stream);
 
 /*
  * kvs_paged_decode_attn for callers that cannot allocate device memory.
@@ -211,6 +227,9 @@ kvs_status kvs_paged_decode_attn(const void *q, const void *k_cache, const void 
  *    scratch than that, i.e. kvs_paged_decode_ws_bytes(...) > the maximum.
  *  - The first call on each device looks up the array's device address
  *    (cudaGetSymbolAddress); make that first call before any stream capture.
+ *    The address is cached with the id of the device's CUDA context; after
+ *    the context is destroyed and rebuilt (cudaDeviceReset) the next call
+ *    looks it up again, so that call too must come before any capture.
  *  - All calls share the array: calls whose kernels overlap on the GPU
  *    (unordered streams, concurrent threads) race and give wrong results.
  *  - Allocates nothing: no cudaMalloc/cudaFree, no allocating library call.
@@ -219,9 +238,9 @@ kvs_status kvs_paged_decode_attn(const void *q, const void *k_cache, const void 
 kvs_status kvs_paged_decode_attn_static(const void *q, const void *k_cache, const void *v_cache,
                                         const int32_t *block_table, const int32_t *num_tokens,
                                         int32_t B, int32_t Hq, int32_t Hkv, int32_t d,
-                                        int32_t block_size, int32_t max_blocks, float scale,
-                                        kvs_dtype dt, void *o, int32_t *dev_status,
-                                        kvs_stream_t stream);
+                                        int32_t block_size, int32_t max_blocks,
+                                        int32_t pool_blocks, float scale, kvs_dtype dt, void *o,
+                                        int32_t *dev_status, kvs_stream_t stream);
 
 /*
  * Eviction-masked causal attention forward over the continuous trace ([T]

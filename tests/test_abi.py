@@ -46,10 +46,16 @@ def test_host_side_argument_errors(built):
     # invalid sizes / NULL pointers are rejected before any launch
     assert L.kvs_compact_block_table(None, None, None, None, 1, 0, 16, 1, None, 0, None, None, None,
                                      None) == kvs.KVS_ERR_INVALID_ARG
-    assert L.kvs_rope_logical(None, 0, None, None, 1, 1, 96, 1e4, 0, None, 1, None, 0, None,
+    assert L.kvs_rope_logical(None, 0, None, None, 1, 1, 96, 1e4, 0, None, 1, 1, None, 0, None,
                               kvs.KVS_F32, None, None) in (kvs.KVS_ERR_INVALID_ARG, kvs.KVS_ERR_UNSUPPORTED)
-    assert L.kvs_paged_decode_attn(None, None, None, None, None, 1, 3, 2, 128, 16, 4, 1.0, kvs.KVS_BF16,
+    assert L.kvs_paged_decode_attn(None, None, None, None, None, 1, 3, 2, 128, 16, 4, 8, 1.0, kvs.KVS_BF16,
                                    None, None, 0, None, None) == kvs.KVS_ERR_INVALID_ARG
+    # the pool size must be positive, and max_blocks * block_size must fit in int32 (the
+    # kernels index live entries with int32)
+    assert L.kvs_paged_decode_attn(None, None, None, None, None, 1, 8, 1, 128, 16, 4, 0, 1.0, kvs.KVS_BF16,
+                                   None, None, 0, None, None) == kvs.KVS_ERR_INVALID_ARG
+    assert L.kvs_paged_decode_attn(None, None, None, None, None, 1, 8, 1, 128, 16, 2**27, 8, 1.0,
+                                   kvs.KVS_BF16, None, None, 0, None, None) == kvs.KVS_ERR_CAPACITY
     m = kvs._TileMaskC()
     m.B, m.N, m.T = 1, 100, 1
     assert L.kvs_masked_attn_fwd(None, None, None, ctypes.byref(m), 1, 100, 4, 1, 96, 1.0, kvs.KVS_BF16,
@@ -68,17 +74,17 @@ def test_product_path_has_no_oracle_import():
 
 
 def _plan_ws(B, Hq, Hkv, d, bs, max_blocks):
-    """The split plan as documented at kvs_paged_decode_ws_bytes: entries per split
-    tps in {1024, 512, 256, 128}, the largest that still gives 148 CTAs when the
-    sequences are half full; partials (d + 2 floats) per (sequence, query head, split)
-    only when a sequence can need more than one split."""
-    max_tok = max_blocks * bs
-    units = B * Hkv
-    tps = 1024
-    while tps > 128 and units * -(-(max_tok // 2) // tps) < 148:
-        tps //= 2
-    splits = max(1, -(-max_tok // tps))
-    return B * Hq * splits * (d + 2) * 4 if splits > 1 else 16
+    """The work split as documented at kvs_paged_decode_ws_bytes: C CTAs, enough that
+    none takes more than 72 chunks of 16 entries when every table is full, rounded up to
+    whole waves of 444 (and no more than the chunks); scratch = 8 (B + 1) bytes of
+    prefix counts (rounded up to 256) + (C + B Hkv) G (d + 2) fp32 partials."""
+    mc = -(-(max_blocks * bs) // 16)
+    tc = B * Hkv * mc
+    c = -(-tc // 72)
+    c = -(-c // 444) * 444
+    c = max(1, min(c, tc))
+    G = Hq // Hkv
+    return -(-(8 * (B + 1)) // 256) * 256 + (c + B * Hkv) * G * (d + 2) * 4
 
 
 @pytest.mark.parametrize("shape", [(64, 32, 8, 128, 16, 2049),   # paged workload

@@ -164,6 +164,63 @@ def test_decode_group_sizes_and_empty(G):
     assert_close(o, want, BF16_TOL, "decode G")
 
 
+@pytest.mark.parametrize("dt,bs", [("bf16", 16), ("bf16", 1), ("bf16", 4), ("f32", 16)])
+def test_decode_skips_block_ids_outside_the_pool(dt, bs):
+    """Block ids < 0 or >= the pool size are reported (KVS_ERR_INVALID_ARG) and their
+    entries left out of the softmax; nothing outside the pool is read. The expected
+    output is the oracle's decode over the same table with those blocks removed."""
+    rng = np.random.default_rng(11 + bs)
+    B, Hkv, G = 3, 2, 4
+    d = 128 if dt == "bf16" else 64
+    tdt = torch.bfloat16 if dt == "bf16" else torch.float32
+    Hq, M = G * Hkv, (1200 + bs - 1) // bs
+    pool = B * M + 5
+    cast = W.round_bf16 if dt == "bf16" else (lambda a: a)
+    kc = cast(rng.standard_normal((pool, Hkv, bs, d)).astype(np.float32))
+    vc = cast(rng.standard_normal((pool, Hkv, bs, d)).astype(np.float32))
+    q = cast(rng.standard_normal((B, Hq, d)).astype(np.float32))
+    bt = rng.permutation(pool)[: B * M].reshape(B, M).astype(np.int32)
+    bad = [(0, 0, -1), (0, M // 2, pool), (1, 3, -7), (2, M - 2, pool + 1000)]
+    for b, i, v in bad:
+        bt[b, i] = v
+    nt = np.full(B, M * bs, np.int32)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    o = host(kvs.kvs_paged_decode_attn(dev(q, tdt), dev(kc, tdt), dev(vc, tdt), dev(bt), dev(nt), bs,
+                                       1 / np.sqrt(d), status=status))
+    torch.cuda.synchronize()
+    assert status.item() == kvs.KVS_ERR_INVALID_ARG
+    assert np.isfinite(o).all()
+    keep = np.full((B, M), -1, np.int32)
+    nt_keep = np.zeros(B, np.int32)
+    for b in range(B):
+        row = [x for x in bt[b] if 0 <= x < pool]
+        keep[b, :len(row)] = row
+        nt_keep[b] = len(row) * bs
+    want = oracle.paged_decode(q, kc, vc, keep, nt_keep, bs, 1 / np.sqrt(d))
+    assert_close(o, want, BF16_TOL if dt == "bf16" else F32_TOL, f"decode without bad blocks {dt} bs={bs}")
+
+
+@pytest.mark.parametrize("dt", ["bf16", "f32"])
+def test_decode_reports_token_counts_past_the_table(dt):
+    """num_tokens beyond max_blocks * block_size is reported and clamped."""
+    rng = np.random.default_rng(5)
+    B, Hkv, Hq, bs, M = 2, 1, 2, 16, 9
+    d = 128 if dt == "bf16" else 64
+    tdt = torch.bfloat16 if dt == "bf16" else torch.float32
+    pool = B * M
+    kc = W.round_bf16(rng.standard_normal((pool, Hkv, bs, d)).astype(np.float32))
+    vc = W.round_bf16(rng.standard_normal((pool, Hkv, bs, d)).astype(np.float32))
+    q = W.round_bf16(rng.standard_normal((B, Hq, d)).astype(np.float32))
+    bt = rng.permutation(pool).reshape(B, M).astype(np.int32)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    o = host(kvs.kvs_paged_decode_attn(dev(q, tdt), dev(kc, tdt), dev(vc, tdt), dev(bt),
+                                       dev(np.array([M * bs + 5, 20], np.int32)), bs, 0.1, status=status))
+    torch.cuda.synchronize()
+    assert status.item() == kvs.KVS_ERR_INVALID_ARG
+    want = oracle.paged_decode(q, kc, vc, bt, np.array([M * bs, 20], np.int32), bs, 0.1)
+    assert_close(o, want, BF16_TOL if dt == "bf16" else F32_TOL, "clamped count")
+
+
 def test_decode_negative_block_id_reports():
     B, Hkv, d, bs = 1, 1, 128, 16
     kc = torch.zeros((4, Hkv, bs, d), dtype=torch.bfloat16, device="cuda")

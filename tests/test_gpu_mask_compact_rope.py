@@ -188,3 +188,35 @@ def test_rope_scatter_into_paged_cache():
         got_k = host(kc[s // bs, :, s % bs])
         assert (np.abs(got_k - want[i]) <= np.abs(want[i]) * 2.0 ** -8 + 1e-6).all()
         assert torch.equal(vc[s // bs, :, s % bs], v[i])
+
+
+def test_rope_scatter_skips_slots_outside_the_cache():
+    """A slot outside [0, pool * block_size) is reported (KVS_ERR_INVALID_ARG) and
+    nothing is written for its row; every other byte of both caches is untouched
+    except the valid rows' slots."""
+    rng = np.random.default_rng(3)
+    pool, H, bs, d = 12, 2, 16, 128
+    n = 8
+    kc = dev(W.round_bf16(rng.standard_normal((pool, H, bs, d)).astype(np.float32)), torch.bfloat16)
+    vc = dev(W.round_bf16(rng.standard_normal((pool, H, bs, d)).astype(np.float32)), torch.bfloat16)
+    k0, v0 = kc.clone(), vc.clone()
+    k = dev(W.round_bf16(rng.standard_normal((n, H, d)).astype(np.float32)), torch.bfloat16)
+    v = dev(W.round_bf16(rng.standard_normal((n, H, d)).astype(np.float32)), torch.bfloat16)
+    lpos = rng.integers(0, 131072, n).astype(np.int32)
+    slots = np.array([5, -1, pool * bs, 17, pool * bs + 100, 2**40, 190, 0], np.int64)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    kvs.kvs_rope_logical(k, dev(lpos), 5e5, out=kc, out_slot=dev(slots), block_size=bs, v=v, v_out=vc,
+                         status=status)
+    torch.cuda.synchronize()
+    assert status.item() == kvs.KVS_ERR_INVALID_ARG
+    valid = [i for i, s in enumerate(slots) if 0 <= s < pool * bs]
+    want = oracle.rope(host(k), lpos, 5e5)
+    touched = torch.zeros((pool, bs), dtype=torch.bool)
+    for i in valid:
+        s = int(slots[i])
+        touched[s // bs, s % bs] = True
+        got = host(kc[s // bs, :, s % bs])
+        assert (np.abs(got - want[i]) <= np.abs(want[i]) * 2.0 ** -8 + 1e-6).all()
+        assert torch.equal(vc[s // bs, :, s % bs], v[i])
+    keep = (~touched).cuda()[:, None, :, None].expand_as(kc)
+    assert torch.equal(kc[keep], k0[keep]) and torch.equal(vc[keep], v0[keep])

@@ -23,7 +23,7 @@ STATIC_MAX = 16 << 20
 def _lib():
     L = kvs.lib()
     vp, i32 = ctypes.c_void_p, ctypes.c_int32
-    L.kvs_paged_decode_attn_static.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
+    L.kvs_paged_decode_attn_static.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32,
                                                ctypes.c_float, i32, vp, vp, vp]
     L.kvs_paged_decode_attn_static.restype = i32
     return L
@@ -34,7 +34,7 @@ def _static_call(q, kc, vc, bt, nt, bs, scale, out, status):
     B, Hq, d = q.shape
     return L.kvs_paged_decode_attn_static(
         q.data_ptr(), kc.data_ptr(), vc.data_ptr(), bt.data_ptr(), nt.data_ptr(), B, Hq, kc.shape[1], d,
-        bs, bt.shape[1], float(scale), kvs.KVS_BF16, out.data_ptr(), status.data_ptr(),
+        bs, bt.shape[1], kc.shape[0], float(scale), kvs.KVS_BF16, out.data_ptr(), status.data_ptr(),
         torch.cuda.current_stream().cuda_stream)
 
 
@@ -67,6 +67,6 @@ def test_static_decode_rejects_oversized_requests():
     t = torch.zeros(1, dtype=torch.bfloat16, device="cuda")
     i = torch.zeros(1, dtype=torch.int32, device="cuda")
     rc = _lib().kvs_paged_decode_attn_static(t.data_ptr(), t.data_ptr(), t.data_ptr(), i.data_ptr(),
-                                            i.data_ptr(), B, Hq, Hkv, d, bs, M, 0.1, kvs.KVS_BF16,
+                                            i.data_ptr(), B, Hq, Hkv, d, bs, M, 1, 0.1, kvs.KVS_BF16,
                                             t.data_ptr(), i.data_ptr(), None)
     assert rc == kvs.KVS_ERR_CAPACITY
