@@ -26,6 +26,32 @@ def dense_mask_eventwise(events, b, N):
     return m
 
 
+def pytest_terminal_summary(terminalreporter):
+    """Parity report of the GPU comparisons: per check family the largest flat
+    max |got - want| next to the largest excess beyond the stored value's
+    rounding (what the assertions bound). Also written as JSON lines to
+    $KVS_PARITY_REPORT when that is set."""
+    gu = sys.modules.get("gpu_util")
+    if gu is None or not gu.REPORT:
+        return
+    fam = {}
+    for what, flat, exc, tol in gu.REPORT:
+        key = what.split(" b")[0].split(" call")[0]
+        f0, e0, t0, n0 = fam.get(key, (0.0, -1e30, tol, 0))
+        fam[key] = (max(f0, flat), max(e0, exc), tol, n0 + 1)
+    tr = terminalreporter
+    tr.write_sep("-", "parity: flat max-abs | excess beyond rounding | tolerance (checks)")
+    for key in sorted(fam):
+        f, e, t, n = fam[key]
+        tr.write_line(f"{key[:48]:48s} {f:10.3g} {e:10.3g} {t:8.2g} ({n})")
+    path = os.environ.get("KVS_PARITY_REPORT")
+    if path:
+        import json
+        with open(path, "w") as fh:
+            for what, flat, exc, tol in gu.REPORT:
+                fh.write(json.dumps({"check": what, "flat_max_abs": flat, "excess": exc, "tol": tol}) + "\n")
+
+
 @pytest.fixture
 def rng():
     return np.random.default_rng(1234)

@@ -16,6 +16,18 @@ F32_TOL = 1e-5       # max-abs, fp32
 BF16_ROUND = 2.0 ** -9
 F32_ROUND = 2.0 ** -24
 GRAD_REL_L2 = 1e-2   # relative L2 on gradients
+# The bf16 path's log-sum-exp is stored in fp32, so it gets no bf16 allowance.
+# Its error is set by the arithmetic of the forward: the row sum adds
+# exponentials with relative error <= 7.5e-5 (the FMA-pipe cubic; ex2.approx is
+# far tighter), which moves ln(sum) by at most 7.5e-5, and the fp32 scores of the
+# bf16 products carry about 1e-4 of accumulated rounding at |<q,k>| ~ 45. 1e-3
+# leaves a factor of five above that sum.
+LSE_TOL = 1e-3
+
+# Every comparison is recorded (check, flat max |got - want|, max excess beyond
+# the stored value's rounding, tolerance) so that a run can report the flat
+# max-abs beside the rounding-aware figure the assertion uses.
+REPORT = []
 
 
 def dev(x, dtype=None):
@@ -58,11 +70,13 @@ def assert_close(got, want, tol, what="", rnd=None):
         rnd = BF16_ROUND if tol == BF16_TOL else (F32_ROUND if tol == F32_TOL else 0.0)
     if not got.size:
         return 0.0
-    excess = np.abs(got - want) - rnd * np.abs(want)
+    diff = np.abs(got - want)
+    excess = diff - rnd * np.abs(want)
     i = np.unravel_index(np.argmax(excess), excess.shape)
     err = float(excess[i])
+    REPORT.append((what, float(diff.max()), err, tol))
     assert err <= tol, (f"{what}: max-abs beyond output rounding {err:.3g} > {tol} "
-                        f"at {i} (got {got[i]:.6g}, want {want[i]:.6g})")
+                        f"at {i} (got {got[i]:.6g}, want {want[i]:.6g}; flat max-abs {diff.max():.3g})")
     return err
 
 
