@@ -79,12 +79,15 @@ __device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
 // t = x + 1.5*2^23 rounds x to the integer n held in the low mantissa bits of t;
 // f = x - n lies in [-1/2, 1/2]; 2^f comes from a cubic fitted for minimum
 // relative error on that interval (eviction_masked_attention_b200/fit_exp2_poly.py;
-// max relative error 1.5e-4 in fp32, far below the 2^-9 of the bf16 P it feeds);
+// max relative error 7.5e-5 for x > -126, far below the 2^-9 of the bf16 P it
+// feeds; 1.5e-4 at the clamp, where the result is ~1e-38);
 // n is added to the exponent field by one integer multiply-add (bits(t) * 2^23
-// wraps to n * 2^23). Arguments below -127 are clamped (result ~1e-38); valid up
-// to x < 128. Each lane is rounded exactly as the scalar sequence would be.
+// wraps to n * 2^23). Arguments below -126 are clamped to -126 (result ~1e-38):
+// with n = -127 a cubic value below 1 would borrow from the sign bit and give a
+// NaN, so n never goes below -126. Valid up to x < 128. Each lane is rounded
+// exactly as the scalar sequence would be.
 __device__ __forceinline__ void exp2_fma_x2(float x0, float x1, float &y0, float &y1) {
-    const uint64_t x = f2_make(fmaxf(x0, -127.f), fmaxf(x1, -127.f));
+    const uint64_t x = f2_make(fmaxf(x0, -126.f), fmaxf(x1, -126.f));
     const uint64_t magic = f2_make(12582912.f, 12582912.f);
     const uint64_t t = f2_add(x, magic);
     const uint64_t f = f2_sub(x, f2_sub(t, magic));
