@@ -289,14 +289,17 @@ struct Fwd2Smem {
     uint8_t q[2][kTileBytes];
     uint8_t k[2][kTileBytes];
     uint8_t v[2][kTileBytes];
-    uint32_t bits[2][128 * 4];  // mask rows of the tile in each V stage (partial tiles)
-    int32_t pid[2];             // partial index of the tile in each V stage (-1: full)
-    uint64_t bar_q, kfull[2], kempty[2], vfull[2], vempty[2], sfull[2], pfull[2], odone[2], fin;
+    // mask rows of tile n (partial tiles) in stage n % 4, loaded with K(n); stage
+    // n % 4 is refilled only after K(n+2)'s stage was released, i.e. after both
+    // softmax groups finished tile n+1 and so tile n
+    uint32_t bits[4][128 * 4];
+    int32_t pid[4];             // partial index of the tile in each bit stage (-1: full)
+    uint64_t bar_q, kfull[2], kempty[2], vfull[2], vempty[2], sfull[2], pfull[2], odone[2], bfull[4], fin;
     uint32_t tmem_base;
     int abort;
 };
 
-__global__ void __launch_bounds__(kFwd2Threads, 1)
+__global__ void __maxnreg__(200)
     k_attn_fwd_tc2(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, kvs_tile_mask m, int32_t Hq,
                    int32_t Hkv, float scale_log2, __nv_bfloat16 *__restrict__ out,
@@ -325,6 +328,7 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
             mbar_init(&S.pfull[i], 128);
             mbar_init(&S.odone[i], 1);
         }
+        for (int i = 0; i < 4; ++i) mbar_init(&S.bfull[i], 1);
         mbar_init(&S.fin, 1);
         S.abort = 0;
         fence_mbar_init();
@@ -357,15 +361,21 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
                 mbar_expect_tx(&S.kfull[s], kTileBytes);
                 tma_load_4d(S.k[s], &tmK, &S.kfull[s], 0, kvh, k0, b);
                 tma_load_4d(S.k[s] + kTileBytes / 2, &tmK, &S.kfull[s], 64, kvh, k0, b);
-                if (n >= 2 && !mbar_wait(&S.vempty[s], ph, abort, status)) break;
-                // the tile's mask metadata travels with its V stage, which is only
-                // released after both heads' softmax finished this tile
+                // the tile's mask rows go out with K, on their own 4-stage barrier, so
+                // the softmax of tile n never waits for V(n)
+                const int bsg = n & 3;
                 const int32_t pid = m.row_pidx[e0 + n];
-                S.pid[s] = pid;
-                mbar_expect_tx(&S.vfull[s], kTileBytes + (pid >= 0 ? 2048u : 0u));
+                S.pid[bsg] = pid;
+                if (pid >= 0) {
+                    mbar_expect_tx(&S.bfull[bsg], 2048u);
+                    bulk_load(S.bits[bsg], m.bits + (int64_t)pid * 512, 2048, &S.bfull[bsg]);
+                } else {
+                    mbar_arrive(&S.bfull[bsg]);
+                }
+                if (n >= 2 && !mbar_wait(&S.vempty[s], ph, abort, status)) break;
+                mbar_expect_tx(&S.vfull[s], kTileBytes);
                 tma_load_4d(S.v[s], &tmV, &S.vfull[s], 0, kvh, k0, b);
                 tma_load_4d(S.v[s] + kTileBytes / 2, &tmV, &S.vfull[s], 64, kvh, k0, b);
-                if (pid >= 0) bulk_load(S.bits[s], m.bits + (int64_t)pid * 512, 2048, &S.vfull[s]);
             }
         }
     } else if (warp == 1) {
@@ -444,37 +454,37 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
                 ok = false;
                 break;
             }
-            if (!__all_sync(0xffffffffu, mbar_wait(&S.vfull[n & 1], (n >> 1) & 1, abort, status))) {
+            if (!__all_sync(0xffffffffu, mbar_wait(&S.bfull[n & 3], (n >> 2) & 1, abort, status))) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            const bool partial = S.pid[n & 1] >= 0;  // same for the whole CTA
+            const bool partial = S.pid[n & 3] >= 0;  // same for the whole CTA
             uint4 bits = make_uint4(~0u, ~0u, ~0u, ~0u);
-            if (partial) bits = *reinterpret_cast<const uint4 *>(&S.bits[n & 1][row * 4]);
+            if (partial) bits = *reinterpret_cast<const uint4 *>(&S.bits[n & 3][row * 4]);
             const uint32_t wb[4] = {bits.x, bits.y, bits.z, bits.w};
-            // pass 1: row maximum of the (masked) raw scores; 8 independent partial
-            // maxima keep the reduction off one serial dependency chain
+            // one pass over S: all 128 columns of this row come into registers with one
+            // TMEM round trip; 8 independent partial maxima keep the reduction off one
+            // serial dependency chain
+            uint32_t r[4][32];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) tmem_ld32(tmem + lane_off + cS + c * 32, r[c]);
+            tmem_ld_wait();
             float mx8[8];
 #pragma unroll
             for (int u = 0; u < 8; ++u) mx8[u] = -INFINITY;
+            if (partial) {
 #pragma unroll
-            for (int hc = 0; hc < 2; ++hc) {
-                uint32_t r0[32], r1[32];
-                tmem_ld32(tmem + lane_off + cS + hc * 64, r0);
-                tmem_ld32(tmem + lane_off + cS + hc * 64 + 32, r1);
-                tmem_ld_wait();
-                if (partial) {
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        if ((wb[2 * hc] >> j) & 1u) mx8[j & 7] = fmaxf(mx8[j & 7], __uint_as_float(r0[j]));
-                        if ((wb[2 * hc + 1] >> j) & 1u) mx8[j & 7] = fmaxf(mx8[j & 7], __uint_as_float(r1[j]));
-                    }
-                } else {
+                for (int c = 0; c < 4; ++c)
 #pragma unroll
                     for (int j = 0; j < 32; ++j)
-                        mx8[j & 7] = max3f(mx8[j & 7], __uint_as_float(r0[j]), __uint_as_float(r1[j]));
-                }
+                        if ((wb[c] >> j) & 1u) mx8[j & 7] = fmaxf(mx8[j & 7], __uint_as_float(r[c][j]));
+            } else {
+#pragma unroll
+                for (int c = 0; c < 4; c += 2)
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        mx8[j & 7] = max3f(mx8[j & 7], __uint_as_float(r[c][j]), __uint_as_float(r[c + 1][j]));
             }
             float mraw = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                                fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
@@ -506,30 +516,25 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
                     tmem_st32(tmem + lane_off + cO + c * 32, o);
                 }
             }
-            // pass 2: P = 2^(s*c - m) as bf16 pairs over the first 64 columns of S
-            // (the two 32-column chunks of a half are read before their 32 packed
-            // columns overwrite the first of them). Half of the exponentials run on
-            // the FMA pipe (exp2_fma), half on the special-function unit.
+            // P = 2^(s*c - m) as bf16 pairs into the first 64 columns of S (all of S is
+            // already in registers). Half of the exponentials run on the FMA pipe
+            // (exp2_fma), half on the special-function unit.
             const float nref = m_run == -INFINITY ? 0.f : -m_run;
             uint64_t lsum2[4];  // four f32x2 partial row sums
 #pragma unroll
             for (int u = 0; u < 4; ++u) lsum2[u] = 0ull;
-#pragma unroll 1
+#pragma unroll
             for (int hc = 0; hc < 2; ++hc) {
-                uint32_t r0[32], r1[32], pk[32];
-                tmem_ld32(tmem + lane_off + cS + hc * 64, r0);
-                tmem_ld32(tmem + lane_off + cS + hc * 64 + 32, r1);
-                tmem_ld_wait();
-                const uint32_t w0 = hc ? wb[2] : wb[0], w1 = hc ? wb[3] : wb[1];
+                uint32_t pk[32];
 #pragma unroll
                 for (int cc = 0; cc < 2; ++cc) {
-                    const uint32_t(&r)[32] = cc ? r1 : r0;
-                    const uint32_t w = cc ? w1 : w0;
+                    const uint32_t(&rr)[32] = r[2 * hc + cc];
+                    const uint32_t w = wb[2 * hc + cc];
 #pragma unroll
                     for (int j = 0; j < 32; j += 4) {
                         float x0, x1, x2, x3, p0, p1;
-                        fma2(__uint_as_float(r[j]), __uint_as_float(r[j + 1]), scale_log2, nref, x0, x1);
-                        fma2(__uint_as_float(r[j + 2]), __uint_as_float(r[j + 3]), scale_log2, nref, x2, x3);
+                        fma2(__uint_as_float(rr[j]), __uint_as_float(rr[j + 1]), scale_log2, nref, x0, x1);
+                        fma2(__uint_as_float(rr[j + 2]), __uint_as_float(rr[j + 3]), scale_log2, nref, x2, x3);
                         exp2_fma_x2(x0, x1, p0, p1);
                         float p2 = ex2(x2), p3 = ex2(x3);
                         if (partial) {
