@@ -54,6 +54,7 @@ def _args():
     p.add_argument("--scale", type=int, default=1, help="divide the trace length (profiling runs)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-per-config", action="store_true")
     return p.parse_args()
 
 
@@ -366,9 +367,9 @@ def _durations(rec):
 
 
 # DRAM traffic of one launch measured by ncu (dram__bytes_read.sum + dram__bytes_write.sum) on the
-# 1/16-scale bs1 workload (profiles/k_attn_tc_bs1_div16.md): kernel -> (bytes of that launch, visible
-# pairs x query heads it processed, sha1 prefix of the kernel sources it was taken with). The bench
-# scales it to its own launch by the pairs processed and reports null once the sources have changed.
+# 1/16-scale bs1 workload: kernel -> (bytes of that launch, visible pairs x query heads it processed,
+# sha1 prefix of the kernel sources it was taken with). The bench scales it to its own launch by the
+# pairs processed and reports null once the sources have changed.
 TRAFFIC = {"dkdv": (1.785179e9 + 57.587456e6, 27713931 * 64, "80065948775d")}
 
 
@@ -390,6 +391,306 @@ def over_ranks(elapsed_ms: float, pairs: float, device):
     p = torch.tensor([pairs], device=device, dtype=torch.float64)
     torch.distributed.all_reduce(p)
     return float(t.item()), float(p.item())
+
+
+# ----------------------------------------------------------------------------- other configurations
+
+def _time_ms(fn, iters: int, warmup: int = 2) -> float:
+    """Mean device time of fn() over iters calls (CUDA events on the current stream)."""
+    for _ in range(warmup):
+        fn()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    a.record()
+    for _ in range(iters):
+        fn()
+    b.record()
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / iters
+
+
+def _attn_config(cid: int, dev, peaks, bwd: bool, scale: int = 1):
+    """Masked forward (and backward) on one replay configuration at full size."""
+    import eviction_masked_attention_b200 as kvs
+
+    cfg = W.CONFIGS[cid] if scale == 1 else W.scaled(W.CONFIGS[cid], scale)
+    B, N, Hq, Hkv, d = cfg.batch, cfg.n_tokens, cfg.hq, cfg.hkv, cfg.d
+    ev = torch.from_numpy(W.make_event_log(cfg)).to(dev)
+    q, k, v, do = W.replay_tensors_device(cfg, device=dev, with_grad=bwd)
+    mask_ws = torch.empty(kvs.lib().kvs_build_tile_mask_ws_bytes(B, N), dtype=torch.uint8, device=dev)
+    mask = kvs.kvs_build_tile_mask(ev, B, N, ws=mask_ws)
+    t_mask = _time_ms(lambda: kvs.kvs_build_tile_mask(ev, B, N, ws=mask_ws), 5)
+    P = float(mask.visible_pairs)
+    o, lse, o_lo = torch.empty_like(q), torch.empty((B, Hq, N), dtype=torch.float32, device=dev), torch.empty_like(q)
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    fwd = lambda: kvs.kvs_masked_attn_fwd(q, k, v, mask, cfg.scale, out=o, lse=lse, out_lo=o_lo, status=st)
+    t_fwd = _time_ms(fwd, 10 if not bwd else 5)
+    out = {"workload": f"cfg{cid}: {B}x{N}, Hq={Hq}, Hkv={Hkv}, d={d}, {len(ev)} events",
+           "visible_pair_fraction": P / (B * N * (N + 1) / 2), "mask_ms": t_mask, "fwd_ms": t_fwd,
+           "fwd_tflops": 4 * d * P * Hq / (t_fwd * 1e-3) / 1e12}
+    if bwd:
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        ws = torch.empty(kvs.lib().kvs_masked_attn_bwd_ws_bytes(B, N, Hq, Hkv, d, kvs.KVS_BF16),
+                         dtype=torch.uint8, device=dev)
+        bw = lambda: kvs.kvs_masked_attn_bwd(q, k, v, o, do, lse, mask, cfg.scale, dq=dq, dk=dk, dv=dv, ws=ws,
+                                             status=st, o_lo=o_lo)
+        t_bwd = _time_ms(bw, 5)
+        out.update({"bwd_ms": t_bwd, "bwd_tflops": 10 * d * P * Hq / (t_bwd * 1e-3) / 1e12,
+                    "fwd_bwd_tflops": 14 * d * P * Hq / ((t_fwd + t_bwd) * 1e-3) / 1e12})
+        tf = out["fwd_bwd_tflops"]
+    else:
+        tf = out["fwd_tflops"]
+    torch.cuda.synchronize()
+    assert st.item() == 0, f"device status {st.item()}"
+    out["frac_bf16_burst"] = tf / float(peaks.get("bf16_tflops", 1590.0))
+    out["frac_bf16_sustained"] = tf / float(peaks.get("bf16_tflops_sustained", 1400.0))
+    return out
+
+
+def _paged_config(dev, peaks):
+    """The paged-generation configuration: 64 sequences on a 131072-block pool of
+    16-token blocks; one compaction step, then decode over the compacted tables.
+    Also decode over the first 1, 2, ..., 64 sequences (tokens/s against live
+    sequences)."""
+    import eviction_masked_attention_b200 as kvs
+
+    cfg = W.CONFIGS[4]
+    st = W.make_paged_state(cfg)
+    B, Hq, Hkv, d, bs = cfg.batch, cfg.hq, cfg.hkv, cfg.d, st.block_size
+    g = torch.Generator(device=dev)
+    g.manual_seed(4004)
+    kc = torch.randn((st.pool_blocks, Hkv, bs, d), generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+    vc = torch.randn((st.pool_blocks, Hkv, bs, d), generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+    q = torch.randn((B, Hq, d), generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+    bt0, bl0 = torch.from_numpy(st.block_table).to(dev), torch.from_numpy(st.block_lpos).to(dev)
+    nb0, nt0 = torch.from_numpy(st.num_blocks).to(dev), torch.from_numpy(st.num_tokens).to(dev)
+    ev = torch.from_numpy(st.events).to(dev)
+    bt, bl, nb, nt = bt0.clone(), bl0.clone(), nb0.clone(), nt0.clone()
+    freed = torch.empty_like(bt)
+    n_freed = torch.empty_like(nb)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def compact():
+        bt.copy_(bt0); bl.copy_(bl0); nb.copy_(nb0); nt.copy_(nt0)
+        kvs.kvs_compact_block_table(bt, bl, nb, nt, bs, st.pool_blocks, ev, freed=freed, n_freed=n_freed,
+                                    status=status)
+
+    t_restore = _time_ms(lambda: (bt.copy_(bt0), bl.copy_(bl0), nb.copy_(nb0), nt.copy_(nt0)), 20)
+    t_compact = _time_ms(compact, 20) - t_restore
+    compact()
+    torch.cuda.synchronize()
+    ntoks = nt.cpu().numpy().astype(np.int64)
+    nblks = nb.cpu().numpy().astype(np.int64)
+    o = torch.empty_like(q)
+
+    def decode_entry(nseq):
+        ws = torch.empty(kvs.lib().kvs_paged_decode_ws_bytes(nseq, Hq, Hkv, d, bs, bt.shape[1]),
+                         dtype=torch.uint8, device=dev)
+        qs, os_, bts, nts = q[:nseq], o[:nseq], bt[:nseq], nt[:nseq]
+        t = _time_ms(lambda: kvs.kvs_paged_decode_attn(qs, kc, vc, bts, nts, bs, cfg.scale, out=os_, ws=ws,
+                                                       status=status), 20, 3)
+        byts = int(ntoks[:nseq].sum()) * Hkv * d * 2 * 2 + 2 * nseq * Hq * d * 2 + int(nblks[:nseq].sum()) * 4
+        gbs = byts / (t * 1e-3) / 1e9
+        return {"seqs": nseq, "ms": t, "bytes": byts, "gbs": gbs, "tokens_per_s": nseq / (t * 1e-3),
+                "frac_hbm_measured": gbs / float(peaks["hbm_gbs"]), "frac_8tbs": gbs / 8000.0}
+
+    full = decode_entry(B)
+    sweep = [decode_entry(n) for n in (1, 2, 4, 8, 16, 32)] + [full]
+    torch.cuda.synchronize()
+    assert status.item() == 0, f"device status {status.item()}"
+    full.update({"workload": f"cfg4: {B} seqs, bs {bs}, pool {st.pool_blocks} blocks, live "
+                             f"{int(ntoks.min())}..{int(ntoks.max())} tokens after compaction "
+                             f"({len(st.events)} events)",
+                 "compact_us": t_compact * 1e3})
+    return full, [{k: e[k] for k in ("seqs", "ms", "gbs", "tokens_per_s")} for e in sweep]
+
+
+def _reprefill_config(dev, scale: int = 1):
+    """Re-prefill against KV-streams on the summary-policy configuration (4 x 65536
+    tokens, budget 16384, each compaction keeps prompt + summary + overlap = 3584):
+    device time of RoPE + forward + backward of the training replay under each
+    schedule (KV-streams: one continuous trace under the eviction mask; re-prefill:
+    every segment re-processes its retained tokens from position 0), and of the
+    generation-side work at the events (re-prefill: a causal forward over the
+    retained tokens; KV-streams: block-table compaction)."""
+    import eviction_masked_attention_b200 as kvs
+    from eviction_masked_attention_b200 import reprefill as R
+
+    cfg = W.CONFIGS[3] if scale == 1 else W.scaled(W.CONFIGS[3], scale)
+    B, N, Hq, Hkv, d = cfg.batch, cfg.n_tokens, cfg.hq, cfg.hkv, cfg.d
+    ev_np = W.make_event_log(cfg)
+    ev = torch.from_numpy(ev_np).to(dev)
+    q_raw, k_raw, v, do = W.replay_tensors_device(cfg, device=dev)
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    L = kvs.lib()
+
+    # KV-streams: the continuous trace
+    lp = torch.arange(N, dtype=torch.int32, device=dev).repeat(B)
+    q, k = torch.empty_like(q_raw), torch.empty_like(k_raw)
+    mask = kvs.kvs_build_tile_mask(ev, B, N)
+    o, lse, o_lo = torch.empty_like(q), torch.empty((B, Hq, N), dtype=torch.float32, device=dev), torch.empty_like(q)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(L.kvs_masked_attn_bwd_ws_bytes(B, N, Hq, Hkv, d, kvs.KVS_BF16), dtype=torch.uint8, device=dev)
+
+    def kv_train():
+        kvs.kvs_rope_logical(q_raw.view(B * N, Hq, d), lp, cfg.theta, out=q.view(B * N, Hq, d))
+        kvs.kvs_rope_logical(k_raw.view(B * N, Hkv, d), lp, cfg.theta, out=k.view(B * N, Hkv, d))
+        kvs.kvs_masked_attn_fwd(q, k, v, mask, cfg.scale, out=o, lse=lse, out_lo=o_lo, status=st)
+        kvs.kvs_masked_attn_bwd(q, k, v, o, do, lse, mask, cfg.scale, dq=dq, dk=dk, dv=dv, ws=ws, status=st,
+                                o_lo=o_lo)
+
+    t_kv = _time_ms(kv_train, 3, 1)
+    pairs_kv = float(mask.visible_pairs)
+    del q, k, o, lse, o_lo, dq, dk, dv, ws, mask
+    torch.cuda.empty_cache()
+
+    # re-prefill: per trace, per segment, a causal sequence at renumbered positions
+    segs, n_reproc = [], 0
+    none = torch.zeros((0, 4), dtype=torch.int32, device=dev)
+    for b in range(B):
+        for sg in R.schedule(ev_np[ev_np[:, 0] == b][:, 1:4], N):
+            n = len(sg.tokens)
+            idx = torch.from_numpy(sg.tokens).to(dev)
+            seg = {"b": b, "idx": idx, "n": n, "r": len(sg.retained),
+                   "lp": torch.from_numpy(sg.positions).to(dev), "mask": kvs.kvs_build_tile_mask(none, 1, n)}
+            for nm, h in (("q", Hq), ("k", Hkv), ("v", Hkv), ("do", Hq), ("o", Hq), ("olo", Hq), ("dq", Hq),
+                          ("dk", Hkv), ("dv", Hkv), ("qr", Hq), ("kr", Hkv)):
+                seg[nm] = torch.empty((1, n, h, d), dtype=torch.bfloat16, device=dev)
+            seg["lse"] = torch.empty((1, Hq, n), dtype=torch.float32, device=dev)
+            seg["ws"] = torch.empty(L.kvs_masked_attn_bwd_ws_bytes(1, n, Hq, Hkv, d, kvs.KVS_BF16),
+                                    dtype=torch.uint8, device=dev)
+            segs.append(seg)
+            n_reproc += len(sg.retained)
+
+    def rp_train():
+        for sg in segs:
+            b, idx, n = sg["b"], sg["idx"], sg["n"]
+            torch.index_select(q_raw[b], 0, idx, out=sg["q"][0])
+            torch.index_select(k_raw[b], 0, idx, out=sg["k"][0])
+            torch.index_select(v[b], 0, idx, out=sg["v"][0])
+            torch.index_select(do[b], 0, idx, out=sg["do"][0])
+            kvs.kvs_rope_logical(sg["q"][0], sg["lp"], cfg.theta, out=sg["qr"][0])
+            kvs.kvs_rope_logical(sg["k"][0], sg["lp"], cfg.theta, out=sg["kr"][0])
+            kvs.kvs_masked_attn_fwd(sg["qr"], sg["kr"], sg["v"], sg["mask"], cfg.scale, out=sg["o"], lse=sg["lse"],
+                                    out_lo=sg["olo"], status=st)
+            kvs.kvs_masked_attn_bwd(sg["qr"], sg["kr"], sg["v"], sg["o"], sg["do"], sg["lse"], sg["mask"],
+                                    cfg.scale, dq=sg["dq"], dk=sg["dk"], dv=sg["dv"], ws=sg["ws"], status=st,
+                                    o_lo=sg["olo"])
+
+    t_rp = _time_ms(rp_train, 3, 1)
+    pairs_rp = float(sum(sg["n"] * (sg["n"] + 1) // 2 for sg in segs))
+
+    # generation side at the events: re-prefill runs a causal forward over the
+    # retained tokens of each new segment; KV-streams compacts the block table
+    pre = [sg for sg in segs if sg["r"] > 0]
+    pre_masks = [kvs.kvs_build_tile_mask(none, 1, sg["r"]) for sg in pre]
+
+    def rp_prefill():
+        for sg, m in zip(pre, pre_masks):
+            r = sg["r"]
+            kvs.kvs_masked_attn_fwd(sg["qr"][:, :r], sg["kr"][:, :r], sg["v"][:, :r], m, cfg.scale,
+                                    out=sg["o"][:, :r], lse=sg["lse_pre"], residual=False, status=st)
+
+    for sg in pre:
+        sg["lse_pre"] = torch.empty((1, Hq, sg["r"]), dtype=torch.float32, device=dev)
+    t_pre = _time_ms(rp_prefill, 3, 1)
+    torch.cuda.synchronize()
+    assert st.item() == 0, f"device status {st.item()}"
+    kept = cfg.prompt + cfg.summary + cfg.overlap
+    n_ev, extra = R.fig3_count(N, cfg.budget, kept)
+    return {"workload": f"cfg3: {B}x{N}, budget {cfg.budget}, kept {kept} per compaction, {len(ev_np)} events",
+            "kvstreams_train_ms": t_kv, "reprefill_train_ms": t_rp, "train_ratio": t_rp / t_kv,
+            "kvstreams_pairs": pairs_kv, "reprefill_pairs": pairs_rp,
+            "tokens_processed": {"kvstreams": B * N, "reprefill": B * N + n_reproc},
+            "reprefill_prefill_ms": t_pre, "reprocessed_tokens": n_reproc,
+            "fig3": {"events_per_trace": n_ev, "reprocessed_per_trace": extra,
+                     "factor_N_over_B_minus_kept": R.fig3_factor(N, cfg.budget, kept)}}
+
+
+def _packed_config(dev, peaks, scale: int = 1):
+    """Packed multi-trace replay: five traces of different lengths and compaction
+    policies (summary at two points, Markovian carry-over, recent turns, oldest
+    turns at 1-token granularity) in one buffer, RoPE at per-trace positions +
+    forward + backward in one call each, against the same traces run one call
+    per trace."""
+    import eviction_masked_attention_b200 as kvs
+    from eviction_masked_attention_b200 import packing
+
+    mix = W.policy_mix(hq=32, hkv=8, div=scale)
+    Hq, Hkv, d = 32, 8, 128
+    lengths = [c.n_tokens for c in mix]
+    evs = [np.asarray(W.make_trace_events(c, 0), np.int64).reshape(-1, 3) for c in mix]
+    cu, ev, lpos = packing.pack(lengths, evs)
+    Nt = int(cu[-1])
+    g = torch.Generator(device=dev)
+    g.manual_seed(6100)
+    rnd = lambda h: torch.randn((1, Nt, h, d), generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+    q_raw, k_raw, v, do = rnd(Hq), rnd(Hkv), rnd(Hkv), rnd(Hq)
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    L = kvs.lib()
+
+    def job(lo, hi, events):
+        n = hi - lo
+        e = torch.from_numpy(events).to(dev)
+        j = {"n": n, "lp": torch.from_numpy(lpos[lo:hi].copy()).to(dev), "mask": kvs.kvs_build_tile_mask(e, 1, n),
+             "q": torch.empty((1, n, Hq, d), dtype=torch.bfloat16, device=dev),
+             "k": torch.empty((1, n, Hkv, d), dtype=torch.bfloat16, device=dev),
+             "o": torch.empty((1, n, Hq, d), dtype=torch.bfloat16, device=dev),
+             "olo": torch.empty((1, n, Hq, d), dtype=torch.bfloat16, device=dev),
+             "lse": torch.empty((1, Hq, n), dtype=torch.float32, device=dev),
+             "dq": torch.empty((1, n, Hq, d), dtype=torch.bfloat16, device=dev),
+             "dk": torch.empty((1, n, Hkv, d), dtype=torch.bfloat16, device=dev),
+             "dv": torch.empty((1, n, Hkv, d), dtype=torch.bfloat16, device=dev),
+             "ws": torch.empty(L.kvs_masked_attn_bwd_ws_bytes(1, n, Hq, Hkv, d, kvs.KVS_BF16),
+                               dtype=torch.uint8, device=dev),
+             "src": (q_raw[:, lo:hi], k_raw[:, lo:hi], v[:, lo:hi].contiguous(), do[:, lo:hi].contiguous())}
+        return j
+
+    def run(j):
+        qs, ks, vs, dos = j["src"]
+        kvs.kvs_rope_logical(qs[0], j["lp"], 5e5, out=j["q"][0])
+        kvs.kvs_rope_logical(ks[0], j["lp"], 5e5, out=j["k"][0])
+        kvs.kvs_masked_attn_fwd(j["q"], j["k"], vs, j["mask"], 1 / np.sqrt(d), out=j["o"], lse=j["lse"],
+                                out_lo=j["olo"], status=st)
+        kvs.kvs_masked_attn_bwd(j["q"], j["k"], vs, j["o"], dos, j["lse"], j["mask"], 1 / np.sqrt(d), dq=j["dq"],
+                                dk=j["dk"], dv=j["dv"], ws=j["ws"], status=st, o_lo=j["olo"])
+
+    packed = job(0, Nt, ev)
+    pairs = float(packed["mask"].visible_pairs)
+    t_packed = _time_ms(lambda: run(packed), 3, 1)
+    del packed
+    torch.cuda.empty_cache()
+    sep = []
+    for b in range(len(mix)):
+        rows = np.concatenate([np.zeros((len(evs[b]), 1), np.int64), evs[b]], axis=1).astype(np.int32)
+        sep.append(job(int(cu[b]), int(cu[b + 1]), rows))
+    t_sep = _time_ms(lambda: [run(j) for j in sep], 3, 1)
+    torch.cuda.synchronize()
+    assert st.item() == 0, f"device status {st.item()}"
+    tf = 14 * d * pairs * Hq / (t_packed * 1e-3) / 1e12
+    return {"workload": "packed: " + ", ".join(f"{c.name} ({c.n_tokens})" for c in mix) +
+                        f"; Hq={Hq}, Hkv={Hkv}, d={d}",
+            "tokens": Nt, "visible_pairs": pairs, "packed_ms": t_packed, "separate_ms": t_sep,
+            "fwd_bwd_tflops": tf, "frac_bf16_sustained": tf / float(peaks.get("bf16_tflops_sustained", 1400.0))}
+
+
+def per_config(dev, peaks, scale: int = 1):
+    """Throughput on the other configurations at 1 GPU, each kernel timed alone
+    with CUDA events: configuration 2 forward, configuration 3 forward + backward
+    (TFLOP/s on visible pairs), configuration 4 paged decode (GB/s)."""
+    out = {"cfg2_fwd": _attn_config(2, dev, peaks, bwd=False, scale=scale)}
+    torch.cuda.empty_cache()
+    out["cfg3_fwd_bwd"] = _attn_config(3, dev, peaks, bwd=True, scale=scale)
+    torch.cuda.empty_cache()
+    out["cfg4_decode"], out["decode_sweep"] = _paged_config(dev, peaks)
+    torch.cuda.empty_cache()
+    out["packed_policy_mix"] = _packed_config(dev, peaks, scale)
+    torch.cuda.empty_cache()
+    rp = _reprefill_config(dev, scale)
+    rp["kvstreams_compact_us_cfg4"] = out["cfg4_decode"]["compact_us"]
+    out["reprefill_vs_kvstreams"] = rp
+    torch.cuda.empty_cache()
+    return out
 
 
 def run_ours(args):
@@ -489,6 +790,10 @@ def run_ours(args):
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()
     if line is not None:
+        if not args.no_per_config:
+            del step
+            torch.cuda.empty_cache()
+            line["per_config"] = per_config(dev, peaks, args.scale)
         print(json.dumps(line), flush=True)
 
 

@@ -1,10 +1,11 @@
 // Compaction-event log -> kill times -> 128x128 tile mask.
 //
 // Follows the trainer replay of "KV-streams: speeding up agentic RL by
-// operating on the KV cache directly" (later tokens are blocked from spans
-// inference had already removed) and Fig. 2(A) of "KV-streams for Efficient
-// Compaction in Agentic Reinforcement Learning" (one continuous trace with an
-// attention mask that reproduces eviction).
+// operating on the KV cache directly" (a query may not attend to a range that
+// an eviction at or before its position removed; the states of retained tokens
+// stay as they were) and Fig. 2(A) of "KV-streams for Efficient Compaction in
+// Agentic Reinforcement Learning" (one continuous trace, masked to reproduce
+// the evictions).
 //
 // Key j is visible from query t iff j <= t < kappa_j. Inside one tile the
 // visible rows of a key column form one interval [lo, hi), which the kernels
