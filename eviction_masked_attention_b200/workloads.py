@@ -108,6 +108,31 @@ CONFIGS = {
 }
 
 
+def policy_mix(hq: int = 32, hkv: int = 8, div: int = 1) -> List[TraceConfig]:
+    """One trace each of the compaction policies of the paper listing's Fig. 2(B) and
+    Table 2 (prompt + summary + overlap, Markovian carry-over of the last tokens only,
+    sliding window of recent turns, oldest turns out with unpadded 1-token granularity),
+    at several (budget, summary, overlap) points and ragged lengths, for packed
+    multi-trace replay. ``div`` shrinks them like :func:`scaled`."""
+    base = dict(batch=1, hq=hq, hkv=hkv, d=128, theta=5e5, block_size=16, dtype="bf16", prompt=1024, pad=16)
+    mix = [
+        TraceConfig(cid=61, name="summary B16k s512 o2048", n_tokens=40960 + 77, budget=16384, summary=512,
+                    overlap=2048, policy="summary", **base),
+        TraceConfig(cid=62, name="summary B8k s256 o1024", n_tokens=24576 + 33, budget=8192, summary=256,
+                    overlap=1024, policy="summary", **base),
+        TraceConfig(cid=63, name="markovian B8k o2048", n_tokens=30720 + 101, budget=8192, summary=0,
+                    overlap=2048, policy="summary", **base),
+        TraceConfig(cid=64, name="recent turns o4096", n_tokens=20480 + 45, turn_min=256, turn_max=2048,
+                    budget=8192, overlap=4096, policy="recent", **base),
+        TraceConfig(cid=65, name="oldest turns bs1", n_tokens=36864 + 13, turn_min=64, turn_max=4096,
+                    budget=16384, target=14336, policy="oldest",
+                    **dict(base, block_size=1, pad=1)),
+    ]
+    if div > 1:
+        mix = [replace(scaled(c, div), n_tokens=max(128, c.n_tokens // div)) for c in mix]
+    return mix
+
+
 def scaled(cfg: TraceConfig, div: int) -> TraceConfig:
     """A smaller twin of a trace config: the logical length, prompt, turn lengths,
     budgets and spans are divided by ``div`` (kept multiples of the padding unit),
