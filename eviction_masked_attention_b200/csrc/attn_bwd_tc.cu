@@ -10,13 +10,14 @@
 // Three launches, no atomics (deterministic):
 //   prep   D and -LSE*log2(e) per (trace, head, row), padded to whole tiles
 //   dK/dV  one CTA per (key tile, kv head, trace); walks the column lists of
-//          the mask for every query head of the group, in items of 64 query
-//          rows. Transposed products S^T = K Q^T and dP^T = V dO^T put one key
-//          per TMEM lane, so P^T and dS^T are written back to TMEM in bf16 and
-//          used as the A operand of dV += P^T dO and dK += dS^T Q. Two TMEM
-//          buffers and two groups of elementwise warps take the items in turn.
-//          Within a tile a key's visible query rows form one interval
-//          (j <= t < kappa_j), so masking needs only kappa_j, not the bit rows.
+//          the mask for every query head of the group, one 128-row query tile
+//          per item. Transposed products S^T = K Q^T and dP^T = V dO^T put one
+//          key per TMEM lane, so P^T and dS^T are written back to TMEM in bf16
+//          and used as the A operand of dV += P^T dO and dK += dS^T Q; the
+//          next item's S^T and dP^T are issued between them so the elementwise
+//          phases overlap tensor work. Within a tile a key's visible query rows
+//          form one interval (j <= t < kappa_j), so masking needs only kappa_j,
+//          not the bit rows.
 //   dQ     one CTA per (query tile, head, trace) over the row lists:
 //          S = Q K^T, dP = dO V^T, dS (bit-masked) to TMEM, dQ += dS K.
 // Warp roles: warp 0 TMA, warp 1 TMEM + MMA issue (the whole warp runs the
@@ -89,31 +90,41 @@ __device__ __forceinline__ void store_row64(__nv_bfloat16 *dst, const uint32_t (
 
 // ---------------------------------------------------------------------- dK / dV
 //
-// An item is (64-row query half-tile, query head of the group); a CTA walks the
-// items of its key tile: for each listed query tile, each head, both halves.
-// TMEM: S^T in two 64-column buffers [0,64) [64,128), dP^T in two more
-// [128,192) [192,256), dV [256,384), dK [384,512). Two groups of four
-// elementwise warps take the items in turn (group = item parity = buffer), so
-// while one group forms P^T and dS^T of item n the tensor core computes S^T and
-// dP^T of item n+1 and the accumulations of item n-1.
+// An item is (128-row query tile of the key tile's column list, query head of
+// the group). TMEM: S^T [0,128) and dP^T [128,256) of the current item, dV
+// [256,384), dK [384,512). The eight elementwise warps split an item's rows in
+// two halves (warp group h takes rows 64h..64h+63, thread = key lane); each
+// writes its P^T (dS^T) as bf16 pairs into the first 32 of its own 64 columns
+// of S^T (dP^T), so neither half overwrites scores the other still reads. Per
+// item the tensor core runs, in issue order,
+//   dV(n) += P^T(n) dO(n), S^T(n+1) = K Q(n+1)^T, dK(n) += dS^T(n) Q(n),
+//   dP^T(n+1) = V dO(n+1)^T
+// (four M=128 N=128 K=128 products): the elementwise phase P^T(n+1) runs while
+// dK(n) and dP^T(n+1) execute, and dS^T(n) while dV(n) and S^T(n+1) execute.
+// Each product that overwrites a TMEM region is issued after the product that
+// reads it (MMAs run in issue order) and after the elementwise warps reported
+// they had read it.
 
 constexpr int kBwdThreads = 320;  // warp 0 TMA, warp 1 MMA, warps 2..9 elementwise
-constexpr int kDkvStages = 4;
-constexpr uint32_t kHalfTile = 64 * 128 * 2;  // 64 rows x 128 dims, bf16
+constexpr int kDkvStages = 2;
 
 struct DkvSmem {
     uint8_t k[kTile];
     uint8_t v[kTile];
-    uint8_t q[kDkvStages][kHalfTile];
-    uint8_t dout[kDkvStages][kHalfTile];
-    float nl2[kDkvStages][64];  // -lse log2(e) of the half-tile rows
-    float dd[kDkvStages][64];
-    int32_t q0[kDkvStages], full_tile[kDkvStages];  // half-tile origin, FULL flag of its tile
-    uint64_t kv_full, full[kDkvStages], empty[kDkvStages], st_full[2], dp_full[2], p_ready[2],
-        ds_ready[2], acc_done, fin;
+    uint8_t q[kDkvStages][kTile];
+    uint8_t dout[kDkvStages][kTile];
+    float nl2[kDkvStages][128];  // -lse log2(e) of the tile's rows
+    float dd[kDkvStages][128];
+    int32_t q0[kDkvStages], full_tile[kDkvStages];  // tile origin, FULL flag
+    uint64_t kv_full, full[kDkvStages], empty[kDkvStages], st_full, dp_full, p_ready, ds_ready,
+        acc_done, fin;
     uint32_t tmem_base;
     int abort;
 };
+
+// TMEM column of the bf16 pairs of rows 16kk..16kk+15 inside a 128-column region
+// whose halves hold rows 0..63 and 64..127 in their first 32 columns.
+__device__ __forceinline__ uint32_t packed_col(int kk) { return kk < 4 ? 8 * kk : 64 + 8 * (kk - 4); }
 
 __global__ void __launch_bounds__(kBwdThreads, 1)
     k_attn_dkdv_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -133,7 +144,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int kvh = rem % Hkv, b = rem / Hkv;
     const int k0 = kj * 128;
     const int32_t c0 = m.col_ptr[b * T + kj], ncol = m.col_ptr[b * T + kj + 1] - c0;
-    const int nw = ncol * G * 2;
+    const int nw = ncol * G;
     if (grid_timed_out(status)) return;
 
     if (threadIdx.x == 0) {
@@ -142,12 +153,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             mbar_init(&S.full[i], 1);
             mbar_init(&S.empty[i], 1);
         }
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(&S.st_full[i], 1);
-            mbar_init(&S.dp_full[i], 1);
-            mbar_init(&S.p_ready[i], 128);
-            mbar_init(&S.ds_ready[i], 128);
-        }
+        mbar_init(&S.st_full, 1);
+        mbar_init(&S.dp_full, 1);
+        mbar_init(&S.p_ready, 256);
+        mbar_init(&S.ds_ready, 256);
         mbar_init(&S.acc_done, 1);
         mbar_init(&S.fin, 1);
         S.abort = 0;
@@ -176,112 +185,98 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 if (n >= kDkvStages &&
                     !mbar_wait(&S.empty[s], ((n / kDkvStages) - 1) & 1, abort, status))
                     break;
-                const int e = n / (2 * G), r = n % (2 * G), h = kvh * G + (r >> 1);
-                const int q0 = m.col_row[c0 + e] * 128 + (r & 1) * 64;
+                const int e = n / G, h = kvh * G + n % G;
+                const int q0 = m.col_row[c0 + e] * 128;
                 S.q0[s] = q0;
                 S.full_tile[s] = m.col_pidx[c0 + e] < 0;
-                mbar_expect_tx(&S.full[s], 2 * kHalfTile + 512);
+                mbar_expect_tx(&S.full[s], 2 * kTile + 1024);
                 tma_load_4d(S.q[s], &tmQ, &S.full[s], 0, h, q0, b);
-                tma_load_4d(S.q[s] + kHalfTile / 2, &tmQ, &S.full[s], 64, h, q0, b);
+                tma_load_4d(S.q[s] + kTile / 2, &tmQ, &S.full[s], 64, h, q0, b);
                 tma_load_4d(S.dout[s], &tmO, &S.full[s], 0, h, q0, b);
-                tma_load_4d(S.dout[s] + kHalfTile / 2, &tmO, &S.full[s], 64, h, q0, b);
+                tma_load_4d(S.dout[s] + kTile / 2, &tmO, &S.full[s], 64, h, q0, b);
                 const int64_t ro = ((int64_t)b * Hq + h) * Tpad + q0;
-                bulk_load(S.nl2[s], NL2 + ro, 256, &S.full[s]);
-                bulk_load(S.dd[s], Drow + ro, 256, &S.full[s]);
+                bulk_load(S.nl2[s], NL2 + ro, 512, &S.full[s]);
+                bulk_load(S.dd[s], Drow + ro, 512, &S.full[s]);
             }
         }
     } else if (warp == 1) {
         if (nw > 0) {
             const bool leader = elect_one();
-            const uint32_t idT = idesc_bf16(128, 64, false, false);   // S^T, dP^T: both K-major
-            const uint32_t idMN = idesc_bf16(128, 128, false, true);  // dV, dK: B MN-major
+            const uint32_t idT = idesc_bf16(128, 128, false, false);   // S^T, dP^T: both K-major
+            const uint32_t idMN = idesc_bf16(128, 128, false, true);   // dV, dK: B MN-major
             const uint64_t kd = sw128_desc(smem_u32(S.k), 16, 1024);
             const uint64_t vd = sw128_desc(smem_u32(S.v), 16, 1024);
             // stage 0 of Q and dO as K-major (B of S^T, dP^T) and MN-major (B of dK, dV)
             const uint64_t qk0 = sw128_desc(smem_u32(S.q[0]), 16, 1024);
             const uint64_t ok0 = sw128_desc(smem_u32(S.dout[0]), 16, 1024);
-            const uint64_t qm0 = sw128_desc(smem_u32(S.q[0]), kHalfTile / 2, 1024);
-            const uint64_t om0 = sw128_desc(smem_u32(S.dout[0]), kHalfTile / 2, 1024);
-            // S^T = K Q^T (issue_st) and dP^T = V dO^T (issue_dp) of item n into buffer n & 1
-            auto issue_st = [&](int n) -> bool {
-                const int s = n % kDkvStages;
-                if (!warp_wait(&S.full[s], (n / kDkvStages) & 1, abort, status)) return false;
+            const uint64_t qm0 = sw128_desc(smem_u32(S.q[0]), kTile / 2, 1024);
+            const uint64_t om0 = sw128_desc(smem_u32(S.dout[0]), kTile / 2, 1024);
+            // S^T = K Q^T and dP^T = V dO^T of item n (its stage already waited for)
+            auto issue_t = [&](int n, uint64_t a, uint64_t b0, uint32_t dst, uint64_t *bar) {
+                const uint64_t bd = desc_add(b0, (n % kDkvStages) * kTile);  // q[s], dout[s]: kTile apart
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t off = (kk >> 2) * (kTile / 2) + (kk & 3) * 32;
+                    if (leader) mma_ss(dst, desc_add(a, off), desc_add(bd, off), idT, kk > 0);
+                }
+                if (leader) mma_commit(bar);
+            };
+            bool ok = warp_wait(&S.kv_full, 0, abort, status) && warp_wait(&S.full[0], 0, abort, status);
+            if (ok) {
                 tc_fence_after();
-                const uint64_t qd = desc_add(qk0, s * kHalfTile);
-                const uint32_t dst = tmem + cST + (uint32_t)(n & 1) * 64;
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t offa = (kk >> 2) * (kTile / 2) + (kk & 3) * 32;
-                    const uint32_t offb = (kk >> 2) * (kHalfTile / 2) + (kk & 3) * 32;
-                    if (leader) mma_ss(dst, desc_add(kd, offa), desc_add(qd, offb), idT, kk > 0);
-                }
-                if (leader) mma_commit(&S.st_full[n & 1]);
-                return true;
-            };
-            auto issue_dp = [&](int n) {  // stage already waited for by issue_st(n)
-                const int s = n % kDkvStages;
-                const uint64_t od = desc_add(ok0, s * kHalfTile);
-                const uint32_t ddp = tmem + cDP + (uint32_t)(n & 1) * 64;
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t offa = (kk >> 2) * (kTile / 2) + (kk & 3) * 32;
-                    const uint32_t offb = (kk >> 2) * (kHalfTile / 2) + (kk & 3) * 32;
-                    if (leader) mma_ss(ddp, desc_add(vd, offa), desc_add(od, offb), idT, kk > 0);
-                }
-                if (leader) mma_commit(&S.dp_full[n & 1]);
-            };
-            bool ok = warp_wait(&S.kv_full, 0, abort, status) && issue_st(0);
-            if (ok) issue_dp(0);
-            if (ok && nw > 1) {
-                ok = issue_st(1);
-                if (ok) issue_dp(1);
+                issue_t(0, kd, qk0, tmem + cST, &S.st_full);
+                issue_t(0, vd, ok0, tmem + cDP, &S.dp_full);
             }
-            // Per item n: dV(n), S^T(n+2), [dS^T(n) ready] dK(n), dP^T(n+2). Item n+2
-            // reuses item n's buffers; every MMA that reads them (dV(n) reads P^T
-            // from the S^T buffer, dK(n) reads dS^T from the dP^T buffer) is issued
-            // before the product that overwrites them, and MMAs run in order. S^T(n+2)
-            // goes ahead of the dS^T wait so the tensor core has work while it is formed.
             for (int n = 0; ok && n < nw; ++n) {
                 const int s = n % kDkvStages;
-                const uint32_t buf = (uint32_t)(n & 1) * 64;
-                const uint64_t qm = desc_add(qm0, s * kHalfTile), om = desc_add(om0, s * kHalfTile);
-                const uint32_t pa = tmem + cST + buf, sa = tmem + cDP + buf, acc = n > 0 ? 1u : 0u;
-                if (!warp_wait(&S.p_ready[n & 1], (n >> 1) & 1, abort, status)) break;
+                const uint64_t qm = desc_add(qm0, s * kTile), om = desc_add(om0, s * kTile);
+                const uint32_t acc = n > 0 ? 1u : 0u;
+                if (!warp_wait(&S.p_ready, n & 1, abort, status)) break;
                 tc_fence_after();
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    if (leader) mma_ts(tmem + cDV, pa + kk * 8, desc_add(om, kk * 2048), idMN, kk > 0 ? 1u : acc);
-                if (n + 2 < nw && !issue_st(n + 2)) break;
-                if (!warp_wait(&S.ds_ready[n & 1], (n >> 1) & 1, abort, status)) break;
+                for (int kk = 0; kk < 8; ++kk)
+                    if (leader)
+                        mma_ts(tmem + cDV, tmem + cST + packed_col(kk), desc_add(om, kk * 2048), idMN,
+                               kk > 0 ? 1u : acc);
+                const bool more = n + 1 < nw;
+                if (more) {
+                    if (!warp_wait(&S.full[(n + 1) % kDkvStages], ((n + 1) / kDkvStages) & 1, abort, status))
+                        break;
+                    tc_fence_after();
+                    issue_t(n + 1, kd, qk0, tmem + cST, &S.st_full);
+                }
+                if (!warp_wait(&S.ds_ready, n & 1, abort, status)) break;
                 tc_fence_after();
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    if (leader) mma_ts(tmem + cDK, sa + kk * 8, desc_add(qm, kk * 2048), idMN, kk > 0 ? 1u : acc);
+                for (int kk = 0; kk < 8; ++kk)
+                    if (leader)
+                        mma_ts(tmem + cDK, tmem + cDP + packed_col(kk), desc_add(qm, kk * 2048), idMN,
+                               kk > 0 ? 1u : acc);
                 if (leader) mma_commit(&S.empty[s]);
-                if (n + 2 < nw) issue_dp(n + 2);
+                if (more) issue_t(n + 1, vd, ok0, tmem + cDP, &S.dp_full);
             }
             if (leader) mma_commit(&S.acc_done);
             if (leader) mma_commit(&S.fin);
             wait_done(&S.fin, 0);
         }
     } else {
-        // thread = key row c (TMEM lane); group = item parity = TMEM buffer
-        const int quad = warp & 3, group = (warp - 2) >> 2;
+        // thread = key row c (TMEM lane); group h takes query rows 64h..64h+63 of each item
+        const int quad = warp & 3, h = (warp - 2) >> 2;
         const int c = quad * 32 + lane;
         const int j = k0 + c;
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-        const uint32_t colS = cST + group * 64, colP = cDP + group * 64;
+        const uint32_t colS = cST + h * 64, colP = cDP + h * 64;
         const int32_t kap = j < N ? m.kappa[(int64_t)b * N + j] : 0;
         bool ok = true;
-        for (int n = group; n < nw; n += 2) {
+        for (int n = 0; n < nw; ++n) {
             const int s = n % kDkvStages;
-            const uint32_t ph = (n >> 1) & 1;
+            const uint32_t ph = n & 1;
             if (!warp_wait(&S.full[s], (n / kDkvStages) & 1, abort, status)) {
                 ok = false;
                 break;
             }
-            const int q0 = S.q0[s];
-            // visible query rows of this key inside the half-tile: [rlo, rhi) (j <= t < kappa_j)
+            const int q0 = S.q0[s] + 64 * h;  // this group's first row
+            // visible query rows of this key among the group's 64: [rlo, rhi) (j <= t < kappa_j)
             int rlo = 0, rhi = 64;
             if (!S.full_tile[s]) {
                 if (j >= N) {
@@ -292,7 +287,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     rhi = (int)(hi < 0 ? 0 : (hi > 64 ? 64 : hi));
                 }
             }
-            if (!warp_wait(&S.st_full[group], ph, abort, status)) {
+            if (!warp_wait(&S.st_full, ph, abort, status)) {
                 ok = false;
                 break;
             }
@@ -305,7 +300,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 tmem_ld32(tmem + lane_off + colS, r0);
                 tmem_ld32(tmem + lane_off + colS + 32, r1);
                 tmem_ld_wait();
-                const float4 *l2v = reinterpret_cast<const float4 *>(S.nl2[s]);
+                const float4 *l2v = reinterpret_cast<const float4 *>(S.nl2[s] + 64 * h);
                 const bool all_vis = rlo <= 0 && rhi >= 64;
                 if (__all_sync(0xffffffffu, all_vis)) {
 #pragma unroll
@@ -344,8 +339,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             }
             tmem_st_wait();
             tc_fence_before();
-            mbar_arrive(&S.p_ready[group]);
-            if (!warp_wait(&S.dp_full[group], ph, abort, status)) {
+            mbar_arrive(&S.p_ready);
+            if (!warp_wait(&S.dp_full, ph, abort, status)) {
                 ok = false;
                 break;
             }
@@ -356,7 +351,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 tmem_ld32(tmem + lane_off + colP, r0);
                 tmem_ld32(tmem + lane_off + colP + 32, r1);
                 tmem_ld_wait();
-                const float4 *ddv = reinterpret_cast<const float4 *>(S.dd[s]);
+                const float4 *ddv = reinterpret_cast<const float4 *>(S.dd[s] + 64 * h);
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
                     const float4 dv4 = ddv[i];
@@ -377,10 +372,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             }
             tmem_st_wait();
             tc_fence_before();
-            mbar_arrive(&S.ds_ready[group]);
+            mbar_arrive(&S.ds_ready);
         }
         // each group writes 64 of the 128 dimensions of dV and dK
-        const uint32_t col0 = group * 64;
+        const uint32_t col0 = h * 64;
         if (ok && nw > 0 && warp_wait(&S.acc_done, 0, abort, status)) {
             tc_fence_after();
             const int64_t ro = (((int64_t)b * N + j) * Hkv + kvh) * 128 + col0;
@@ -416,20 +411,23 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 // current ones, so the tensor core computes them while dS is being formed.
 
 // K is needed from S_n until dQ_n, at the end of the item, V only for dP_n. K
-// therefore has three stages (the load of K_{n+1} overlaps item n instead of
-// waiting for dQ_{n-1}), V one: V_{n+1} loads while the elementwise warps form
-// P_n, long before dP_{n+1} is issued.
+// has three stages, so the load of K_{n+1} goes out when dQ_{n-2} completes,
+// an item ahead of S_{n+1}; V has two, so V_{n+1} goes out when dP_{n-1}
+// completes, four products ahead of dP_{n+1}. (With one V stage the load of
+// V_{n+1} waited for dP_n, only S_{n+1} ahead of its use.) The mask rows of a
+// partial tile are read by each elementwise thread from global memory (L2)
+// while it waits for S_n: there is no shared memory left for them.
 constexpr int kDqKStages = 3;
+constexpr int kDqVStages = 2;
 
 struct DqSmem {
     uint8_t q[kTile];
     uint8_t dout[kTile];
     uint8_t k[kDqKStages][kTile];
-    uint8_t v[kTile];
-    uint32_t bits[kDqKStages][128 * 4];  // mask rows of the key tile in each K stage (partial tiles)
-    int32_t pid[kDqKStages];             // its partial index (-1: full)
-    uint64_t qo_full, kfull[kDqKStages], kempty[kDqKStages], vfull, vempty, s_full, dp_full, s_free,
-        dp_free, ds_ready, dq_done, acc_done, fin;
+    uint8_t v[kDqVStages][kTile];
+    int32_t pid[kDqKStages];  // partial index of the key tile in each K stage (-1: full)
+    uint64_t qo_full, kfull[kDqKStages], kempty[kDqKStages], vfull[kDqVStages], vempty[kDqVStages], s_full,
+        dp_full, s_free, dp_free, ds_ready, dq_done, acc_done, fin;
     uint32_t tmem_base;
     int abort;
 };
@@ -459,8 +457,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             mbar_init(&S.kfull[i], 1);
             mbar_init(&S.kempty[i], 1);
         }
-        mbar_init(&S.vfull, 1);
-        mbar_init(&S.vempty, 1);
+        for (int i = 0; i < kDqVStages; ++i) {
+            mbar_init(&S.vfull[i], 1);
+            mbar_init(&S.vempty[i], 1);
+        }
         mbar_init(&S.s_full, 1);
         mbar_init(&S.dp_full, 1);
         mbar_init(&S.s_free, 256);
@@ -496,16 +496,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 if (n >= kDqKStages &&
                     !mbar_wait(&S.kempty[ks], ((n / kDqKStages) - 1) & 1, abort, status))
                     break;
-                const int32_t pid = m.row_pidx[e0 + n];
-                S.pid[ks] = pid;
-                mbar_expect_tx(&S.kfull[ks], kTile + (pid >= 0 ? 2048u : 0u));
+                S.pid[ks] = m.row_pidx[e0 + n];
+                mbar_expect_tx(&S.kfull[ks], kTile);
                 tma_load_4d(S.k[ks], &tmK, &S.kfull[ks], 0, kvh, k0, b);
                 tma_load_4d(S.k[ks] + kTile / 2, &tmK, &S.kfull[ks], 64, kvh, k0, b);
-                if (pid >= 0) bulk_load(S.bits[ks], m.bits + (int64_t)pid * 512, 2048, &S.kfull[ks]);
-                if (n >= 1 && !mbar_wait(&S.vempty, (n - 1) & 1, abort, status)) break;
-                mbar_expect_tx(&S.vfull, kTile);
-                tma_load_4d(S.v, &tmV, &S.vfull, 0, kvh, k0, b);
-                tma_load_4d(S.v + kTile / 2, &tmV, &S.vfull, 64, kvh, k0, b);
+                const int vs = n % kDqVStages;
+                if (n >= kDqVStages &&
+                    !mbar_wait(&S.vempty[vs], ((n / kDqVStages) - 1) & 1, abort, status))
+                    break;
+                mbar_expect_tx(&S.vfull[vs], kTile);
+                tma_load_4d(S.v[vs], &tmV, &S.vfull[vs], 0, kvh, k0, b);
+                tma_load_4d(S.v[vs] + kTile / 2, &tmV, &S.vfull[vs], 64, kvh, k0, b);
             }
         }
     } else if (warp == 1) {
@@ -517,7 +518,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             const uint64_t od = sw128_desc(smem_u32(S.dout), 16, 1024);
             const uint64_t kd0 = sw128_desc(smem_u32(S.k[0]), 16, 1024);         // + stage * kTile
             const uint64_t km0 = sw128_desc(smem_u32(S.k[0]), kTile / 2, 1024);  // MN-major view
-            const uint64_t vd = sw128_desc(smem_u32(S.v), 16, 1024);
+            const uint64_t vd0 = sw128_desc(smem_u32(S.v[0]), 16, 1024);  // + stage * kTile
             auto issue_s_dp = [&](int n) -> bool {
                 const int ks = n % kDqKStages;
                 if (!warp_wait(&S.kfull[ks], (n / kDqKStages) & 1, abort, status)) return false;
@@ -531,15 +532,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 }
                 if (leader) mma_commit(&S.s_full);
                 if (n > 0 && !warp_wait(&S.dp_free, (n - 1) & 1, abort, status)) return false;
-                if (!warp_wait(&S.vfull, n & 1, abort, status)) return false;
+                const int vs = n % kDqVStages;
+                if (!warp_wait(&S.vfull[vs], (n / kDqVStages) & 1, abort, status)) return false;
                 tc_fence_after();
+                const uint64_t vd = desc_add(vd0, vs * kTile);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint32_t off = (kk >> 2) * (kTile / 2) + (kk & 3) * 32;
                     if (leader) mma_ss(tmem + cDP, desc_add(od, off), desc_add(vd, off), idKM, kk > 0);
                 }
                 if (leader) mma_commit(&S.dp_full);
-                if (leader) mma_commit(&S.vempty);
+                if (leader) mma_commit(&S.vempty[vs]);
                 return true;
             };
             bool ok = warp_wait(&S.qo_full, 0, abort, status) && issue_s_dp(0);
@@ -573,21 +576,23 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         bool ok = true;
         for (int n = 0; n < nt; ++n) {
             const int s = n & 1;
-            if (!warp_wait(&S.s_full, n & 1, abort, status)) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
-            // the K stage carries the tile's mask rows; it is refilled only after
-            // dQ_n, i.e. after this item's dS
+            // the K stage carries the tile's partial index; it is refilled only after
+            // dQ_n, i.e. after this item's dS. The mask row comes from global memory,
+            // requested before the wait for S_n.
             const int ks = n % kDqKStages;
             if (!warp_wait(&S.kfull[ks], (n / kDqKStages) & 1, abort, status)) {
                 ok = false;
                 break;
             }
-            const bool partial = S.pid[ks] >= 0;  // same for the whole CTA
+            const int32_t pid = S.pid[ks];
+            const bool partial = pid >= 0;  // same for the whole CTA
             uint2 bits = make_uint2(~0u, ~0u);
-            if (partial) bits = *reinterpret_cast<const uint2 *>(&S.bits[ks][row * 4 + half * 2]);
+            if (partial) bits = *reinterpret_cast<const uint2 *>(m.bits + (int64_t)pid * 512 + row * 4 + half * 2);
+            if (!warp_wait(&S.s_full, n & 1, abort, status)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
             // P = 2^(S c - LSE log2 e) for this thread's 64 key columns, kept as bf16
             // pairs; dS = P (dP - D) then rounds to bf16 for the dQ MMA
             uint32_t pp[32];
@@ -688,10 +693,9 @@ cudaError_t launch_bwd_tc(const void *q, const void *k, const void *v, const voi
                           const void *o_lo, const void *dO, const float *lse, const kvs_tile_mask &m, int32_t Hq,
                           int32_t Hkv, float scale, void *dq, void *dk, void *dv, void *ws,
                           int32_t stages, int32_t *status, cudaStream_t s, bool *map_ok) {
-    CUtensorMap tq, tk, tv, to, tq64, to64;
+    CUtensorMap tq, tk, tv, to;
     *map_ok = make_tmap_bnhd(&tq, q, m.B, m.N, Hq, 128) && make_tmap_bnhd(&tk, k, m.B, m.N, Hkv, 128) &&
-              make_tmap_bnhd(&tv, v, m.B, m.N, Hkv, 128) && make_tmap_bnhd(&to, dO, m.B, m.N, Hq, 128) &&
-              make_tmap_bnhd(&tq64, q, m.B, m.N, Hq, 64) && make_tmap_bnhd(&to64, dO, m.B, m.N, Hq, 64);
+              make_tmap_bnhd(&tv, v, m.B, m.N, Hkv, 128) && make_tmap_bnhd(&to, dO, m.B, m.N, Hq, 128);
     if (!*map_ok) return cudaSuccess;
     const int32_t Tpad = m.T * 128;
     float *Drow = (float *)ws;
@@ -709,7 +713,7 @@ cudaError_t launch_bwd_tc(const void *q, const void *k, const void *v, const voi
                                  (int)smem);
         if (e != cudaSuccess) return e;
         k_attn_dkdv_tc<<<(unsigned)((int64_t)m.B * Hkv * m.T), kBwdThreads, smem, s>>>(
-            tq64, tk, tv, to64, m, Hq, Hkv, scale, sl2, Drow, NL2, (__nv_bfloat16 *)dk,
+            tq, tk, tv, to, m, Hq, Hkv, scale, sl2, Drow, NL2, (__nv_bfloat16 *)dk,
             (__nv_bfloat16 *)dv, status);
     }
     if (stages & KVS_BWD_DQ) {
