@@ -299,7 +299,7 @@ struct Fwd2Smem {
     int abort;
 };
 
-__global__ void __maxnreg__(200)
+__global__ void __launch_bounds__(kFwd2Threads, 1)
     k_attn_fwd_tc2(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, kvs_tile_mask m, int32_t Hq,
                    int32_t Hkv, float scale_log2, __nv_bfloat16 *__restrict__ out,
@@ -463,28 +463,28 @@ __global__ void __maxnreg__(200)
             uint4 bits = make_uint4(~0u, ~0u, ~0u, ~0u);
             if (partial) bits = *reinterpret_cast<const uint4 *>(&S.bits[n & 3][row * 4]);
             const uint32_t wb[4] = {bits.x, bits.y, bits.z, bits.w};
-            // one pass over S: all 128 columns of this row come into registers with one
-            // TMEM round trip; 8 independent partial maxima keep the reduction off one
-            // serial dependency chain
-            uint32_t r[4][32];
-#pragma unroll
-            for (int c = 0; c < 4; ++c) tmem_ld32(tmem + lane_off + cS + c * 32, r[c]);
-            tmem_ld_wait();
+            // pass 1: row maximum of the (masked) raw scores; 8 independent partial
+            // maxima keep the reduction off one serial dependency chain
             float mx8[8];
 #pragma unroll
             for (int u = 0; u < 8; ++u) mx8[u] = -INFINITY;
-            if (partial) {
 #pragma unroll
-                for (int c = 0; c < 4; ++c)
+            for (int hc = 0; hc < 2; ++hc) {
+                uint32_t r0[32], r1[32];
+                tmem_ld32(tmem + lane_off + cS + hc * 64, r0);
+                tmem_ld32(tmem + lane_off + cS + hc * 64 + 32, r1);
+                tmem_ld_wait();
+                if (partial) {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        if ((wb[2 * hc] >> j) & 1u) mx8[j & 7] = fmaxf(mx8[j & 7], __uint_as_float(r0[j]));
+                        if ((wb[2 * hc + 1] >> j) & 1u) mx8[j & 7] = fmaxf(mx8[j & 7], __uint_as_float(r1[j]));
+                    }
+                } else {
 #pragma unroll
                     for (int j = 0; j < 32; ++j)
-                        if ((wb[c] >> j) & 1u) mx8[j & 7] = fmaxf(mx8[j & 7], __uint_as_float(r[c][j]));
-            } else {
-#pragma unroll
-                for (int c = 0; c < 4; c += 2)
-#pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        mx8[j & 7] = max3f(mx8[j & 7], __uint_as_float(r[c][j]), __uint_as_float(r[c + 1][j]));
+                        mx8[j & 7] = max3f(mx8[j & 7], __uint_as_float(r0[j]), __uint_as_float(r1[j]));
+                }
             }
             float mraw = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                                fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
@@ -516,25 +516,30 @@ __global__ void __maxnreg__(200)
                     tmem_st32(tmem + lane_off + cO + c * 32, o);
                 }
             }
-            // P = 2^(s*c - m) as bf16 pairs into the first 64 columns of S (all of S is
-            // already in registers). Half of the exponentials run on the FMA pipe
-            // (exp2_fma), half on the special-function unit.
+            // pass 2: P = 2^(s*c - m) as bf16 pairs over the first 64 columns of S
+            // (the two 32-column chunks of a half are read before their 32 packed
+            // columns overwrite the first of them). Half of the exponentials run on
+            // the FMA pipe (exp2_fma), half on the special-function unit.
             const float nref = m_run == -INFINITY ? 0.f : -m_run;
             uint64_t lsum2[4];  // four f32x2 partial row sums
 #pragma unroll
             for (int u = 0; u < 4; ++u) lsum2[u] = 0ull;
-#pragma unroll
+#pragma unroll 1
             for (int hc = 0; hc < 2; ++hc) {
-                uint32_t pk[32];
+                uint32_t r0[32], r1[32], pk[32];
+                tmem_ld32(tmem + lane_off + cS + hc * 64, r0);
+                tmem_ld32(tmem + lane_off + cS + hc * 64 + 32, r1);
+                tmem_ld_wait();
+                const uint32_t w0 = hc ? wb[2] : wb[0], w1 = hc ? wb[3] : wb[1];
 #pragma unroll
                 for (int cc = 0; cc < 2; ++cc) {
-                    const uint32_t(&rr)[32] = r[2 * hc + cc];
-                    const uint32_t w = wb[2 * hc + cc];
+                    const uint32_t(&r)[32] = cc ? r1 : r0;
+                    const uint32_t w = cc ? w1 : w0;
 #pragma unroll
                     for (int j = 0; j < 32; j += 4) {
                         float x0, x1, x2, x3, p0, p1;
-                        fma2(__uint_as_float(rr[j]), __uint_as_float(rr[j + 1]), scale_log2, nref, x0, x1);
-                        fma2(__uint_as_float(rr[j + 2]), __uint_as_float(rr[j + 3]), scale_log2, nref, x2, x3);
+                        fma2(__uint_as_float(r[j]), __uint_as_float(r[j + 1]), scale_log2, nref, x0, x1);
+                        fma2(__uint_as_float(r[j + 2]), __uint_as_float(r[j + 3]), scale_log2, nref, x2, x3);
                         exp2_fma_x2(x0, x1, p0, p1);
                         float p2 = ex2(x2), p3 = ex2(x3);
                         if (partial) {
