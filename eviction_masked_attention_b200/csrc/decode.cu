@@ -292,12 +292,17 @@ __global__ void __launch_bounds__(D)
     const int64_t c_first = dec_cta_of(cs, tc, n_cta), c_last = dec_cta_of(cs + nch - 1, tc, n_cta);
     if (c_first == c_last) return;  // one piece: written by its CTA
     const int64_t u = (int64_t)b * Hkv + kvh;
+    // CTAs between c_first and c_last whose chunk range is empty (more CTAs than
+    // chunks) wrote nothing: skip them
+    auto empty = [&](int64_t c) { return c * tc / n_cta == (c + 1) * tc / n_cta; };
     float M = -INFINITY;
-    for (int64_t c = c_first; c <= c_last; ++c) M = fmaxf(M, partials[((c + u) * G + g) * (D + 2) + D]);
+    for (int64_t c = c_first; c <= c_last; ++c)
+        if (!empty(c)) M = fmaxf(M, partials[((c + u) * G + g) * (D + 2) + D]);
     const float Mr = M == -INFINITY ? 0.f : M;
     float L = 0.f, A = 0.f;
 #pragma unroll 4
     for (int64_t c = c_first; c <= c_last; ++c) {
+        if (empty(c)) continue;
         const float *pp = partials + ((c + u) * G + g) * (D + 2);
         const float f = ex2(pp[D] - Mr);
         L += pp[D + 1] * f;
