@@ -277,10 +277,11 @@ class Step:
         self.new_slot = torch.tensor([perm[B * N + b].item() for b in range(B)], dtype=torch.int64,
                                      device=dev)
         self.new_lpos = torch.tensor(self.tau, dtype=torch.int32, device=dev)
-        idx = torch.tensor(self.tau, device=dev, dtype=torch.long)
-        self.q_new = self.q_raw[torch.arange(B, device=dev), idx].contiguous()       # [B, Hq, d]
-        self.k_new = self.k_raw[torch.arange(B, device=dev), idx].contiguous()       # [B, Hkv, d]
-        self.v_new = self.v[torch.arange(B, device=dev), idx].contiguous()
+        # rows of the token each trace generates next (gathered from this step's inputs)
+        self.new_rows = torch.tensor([b * N + t for b, t in enumerate(self.tau)], device=dev, dtype=torch.long)
+        self.q_new = torch.empty((B, Hq, d), dtype=self.q_raw.dtype, device=dev)
+        self.k_new = torch.empty((B, Hkv, d), dtype=self.q_raw.dtype, device=dev)
+        self.v_new = torch.empty((B, Hkv, d), dtype=self.q_raw.dtype, device=dev)
         self.q_new_r = torch.empty_like(self.q_new)
         self.o_dec = torch.empty_like(self.q_new)
         L = kvs.lib()
@@ -331,6 +332,9 @@ class Step:
         self.bl.copy_(self.bl0)
         self.nb.copy_(self.nb0)
         self.nt.copy_(self.nb0)
+        torch.index_select(self.q_raw.view(B * N, Hq, d), 0, self.new_rows, out=self.q_new)
+        torch.index_select(self.k_raw.view(B * N, Hkv, d), 0, self.new_rows, out=self.k_new)
+        torch.index_select(self.v.view(B * N, Hkv, d), 0, self.new_rows, out=self.v_new)
         mark("restore")
         kvs.kvs_compact_block_table(self.bt, self.bl, self.nb, self.nt, 1, self.pool, self.gen_events,
                                     freed=self.freed, n_freed=self.n_freed, status=self.status)
@@ -797,41 +801,69 @@ def run_ours(args):
         print(json.dumps(line), flush=True)
 
 
+IN_NAMES = ("q_raw", "k_raw", "v", "do", "events")     # a step's inputs
+OUT_NAMES = ("dq_raw", "dk_raw", "dv", "o_dec")          # a step's results
+
+
 def _e2e(step, args, flops_step):
-    """Inputs (raw q, k, v, dO, event log) copied from pinned host memory every
-    step and the results (dq, dk, dv in the pre-RoPE basis, decode output) read
-    back; timed with CUDA events around copies + step."""
-    ins = [step.q_raw, step.k_raw, step.v, step.do, step.events]
-    outs = [step.dq_raw, step.dk_raw, step.dv, step.o_dec]
+    """Every step copies its inputs (raw q, k, v, dO, event log) from pinned host
+    memory and reads its results (dq, dk in the pre-RoPE basis, dv, the decode
+    output) back, timed with CUDA events from the first copy in to the last copy
+    out. Steps are pipelined as a serving or training loop would run them: two
+    sets of device inputs and results, the copy of step i+1's inputs on one copy
+    stream and of step i-1's results on another while step i computes; a set is
+    refilled only after the step that read it has finished."""
+    ins = [getattr(step, n) for n in IN_NAMES]
+    outs = [getattr(step, n) for n in OUT_NAMES]
     h_in = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in ins]
     h_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs]
     for h, t in zip(h_in, ins):
         h.copy_(t)
-    n = max(1, min(args.steps, 3))
+    sets = [(ins, outs), ([torch.empty_like(t) for t in ins], [torch.empty_like(t) for t in outs])]
+    n = max(3, min(args.steps, 5))
+    comp = torch.cuda.current_stream()
+    h2d, d2h = torch.cuda.Stream(), torch.cuda.Stream()
+    ev = lambda: torch.cuda.Event()
+    in_ready, in_free, out_ready, out_free = [ev(), ev()], [ev(), ev()], [ev(), ev()], [ev(), ev()]
     s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
-    s.record()
-    for _ in range(n):
-        for h, t in zip(h_in, ins):
-            t.copy_(h, non_blocking=True)
+    s.record(h2d)
+    for i in range(n):
+        k = i % 2
+        s_in, s_out = sets[k]
+        with torch.cuda.stream(h2d):
+            if i >= 2:
+                h2d.wait_event(in_free[k])
+            for h, t in zip(h_in, s_in):
+                t.copy_(h, non_blocking=True)
+            in_ready[k].record(h2d)
+        comp.wait_event(in_ready[k])
+        if i >= 2:
+            comp.wait_event(out_free[k])
+        for nm, t in zip(IN_NAMES + OUT_NAMES, s_in + s_out):
+            setattr(step, nm, t)
         step.run()
-        for h, t in zip(h_out, outs):
-            h.copy_(t, non_blocking=True)
-    e.record()
+        in_free[k].record(comp)
+        out_ready[k].record(comp)
+        with torch.cuda.stream(d2h):
+            d2h.wait_event(out_ready[k])
+            for h, t in zip(h_out, s_out):
+                h.copy_(t, non_blocking=True)
+            out_free[k].record(d2h)
+    e.record(d2h)
     torch.cuda.synchronize()
+    for nm, t in zip(IN_NAMES + OUT_NAMES, ins + outs):
+        setattr(step, nm, t)
     ms = s.elapsed_time(e) / n
     world = int(os.environ.get("WORLD_SIZE", "1"))
     if world > 1:
         t = torch.tensor([ms], device=step.dev)
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         ms = float(t.item())
-        flops_all = flops_step  # already the all-rank total
-    else:
-        flops_all = flops_step
-    return {"value": flops_all / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+    return {"value": flops_step / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
             "h2d_bytes_per_step": int(sum(t.numel() * t.element_size() for t in ins)),
             "d2h_bytes_per_step": int(sum(t.numel() * t.element_size() for t in outs)),
-            "ms_per_step": ms, "steps": n}
+            "ms_per_step": ms, "steps": n, "pipelined": "copies of step i+1 in and i-1 out overlap step i"}
 
 
 def main():
