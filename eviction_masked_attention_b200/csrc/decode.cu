@@ -75,15 +75,15 @@ __global__ void __launch_bounds__(kDecThreads)
     const int ktok = lane >> 1, khalf = lane & 1;    // key phase: entry, half row
     const int vpiece = lane & 15, vpar = lane >> 4;  // value phase: 16-B piece, entry parity
     int32_t b = rg.b0;
-    int64_t pre = rg.pre_b0;
+    int32_t pre = rg.pre_b0;
     int32_t ntok = dec_ntok(num_tokens, b, cap);
-    int64_t nch = dec_nch(ntok);
-    int32_t kvh = (int32_t)((rg.x0 - (int64_t)Hkv * pre) / nch);
+    int32_t nch = dec_nch(ntok);
+    int32_t kvh = (rg.x0 - Hkv * pre) / nch;
     for (;;) {
-        const int64_t cs = (int64_t)Hkv * pre + (int64_t)kvh * nch, ce = cs + nch;
-        const int64_t ps = max(rg.x0, cs), pe = min(rg.x1, ce);
-        const int32_t t_begin = (int32_t)((ps - cs) * kDecChunk);
-        const int32_t t_end = min(ntok, (int32_t)((pe - cs) * kDecChunk));
+        const int32_t cs = Hkv * pre + kvh * nch, ce = cs + nch;
+        const int32_t ps = max(rg.x0, cs), pe = min(rg.x1, ce);
+        const int32_t t_begin = (ps - cs) * kDecChunk;
+        const int32_t t_end = min(ntok, (pe - cs) * kDecChunk);
         const bool whole = ps == cs && pe == ce;
         for (int i = threadIdx.x; i < G * D; i += blockDim.x) {
             const int g = i / D, e = i % D;
@@ -292,18 +292,19 @@ __global__ void __launch_bounds__(D)
     const int64_t c_first = dec_cta_of(cs, tc, n_cta), c_last = dec_cta_of(cs + nch - 1, tc, n_cta);
     if (c_first == c_last) return;  // one piece: written by its CTA
     const int64_t u = (int64_t)b * Hkv + kvh;
-    // CTAs between c_first and c_last whose chunk range is empty (more CTAs than
-    // chunks) wrote nothing: skip them
-    auto empty = [&](int64_t c) { return c * tc / n_cta == (c + 1) * tc / n_cta; };
+    // With at least as many chunks as CTAs every CTA in [c_first, c_last] holds a
+    // piece of the unit. With fewer, each CTA holds at most one chunk, and the
+    // unit's pieces are the CTAs of its chunks.
+    const bool per_chunk = tc < n_cta;
+    const int64_t n_it = per_chunk ? nch : c_last - c_first + 1;
+    auto slot = [&](int64_t i) { return (per_chunk ? dec_cta_of(cs + i, tc, n_cta) : c_first + i) + u; };
     float M = -INFINITY;
-    for (int64_t c = c_first; c <= c_last; ++c)
-        if (!empty(c)) M = fmaxf(M, partials[((c + u) * G + g) * (D + 2) + D]);
+    for (int64_t i = 0; i < n_it; ++i) M = fmaxf(M, partials[(slot(i) * G + g) * (D + 2) + D]);
     const float Mr = M == -INFINITY ? 0.f : M;
     float L = 0.f, A = 0.f;
 #pragma unroll 4
-    for (int64_t c = c_first; c <= c_last; ++c) {
-        if (empty(c)) continue;
-        const float *pp = partials + ((c + u) * G + g) * (D + 2);
+    for (int64_t i = 0; i < n_it; ++i) {
+        const float *pp = partials + (slot(i) * G + g) * (D + 2);
         const float f = ex2(pp[D] - Mr);
         L += pp[D + 1] * f;
         A += pp[e] * f;
@@ -355,7 +356,9 @@ extern "C" kvs_status kvs_paged_decode_attn(const void *q, const void *k_cache, 
     if (G != 1 && G != 2 && G != 4 && G != 8) return KVS_ERR_UNSUPPORTED;
     const DecodePlan p = decode_plan(B, Hq, Hkv, d, block_size, max_blocks);
     if (ws_bytes < p.ws_bytes) return KVS_ERR_CAPACITY;
-    if (p.ctas > INT32_MAX) return KVS_ERR_CAPACITY;
+    // chunk coordinates are 32-bit on the device
+    if (p.units * (((int64_t)max_blocks * block_size + kDecChunk - 1) / kDecChunk) > INT32_MAX)
+        return KVS_ERR_CAPACITY;
     int64_t *pre = reinterpret_cast<int64_t *>(static_cast<char *>(ws) + p.pre_off);
     float *part = reinterpret_cast<float *>(static_cast<char *>(ws) + p.part_off);
     const float qs = scale * 1.4426950408889634f;  // base-2 logits

@@ -101,77 +101,17 @@ __global__ void __launch_bounds__(kDmThreads, 3)
     const int g = lane >> 2, t4 = lane & 3;
 
     int32_t b = rg.b0;
-    int64_t pre = rg.pre_b0;
+    int32_t pre = rg.pre_b0;
     int32_t ntok = dec_ntok(num_tokens, b, cap);
-    int64_t nch = dec_nch(ntok);
-    int32_t kvh = (int32_t)((rg.x0 - (int64_t)Hkv * pre) / nch);
+    int32_t nch = dec_nch(ntok);
+    int32_t kvh = (rg.x0 - Hkv * pre) / nch;
     for (;;) {
         // this piece: unit (b, kvh), chunks [ps, pe) of the unit's [cs, ce)
-        const int64_t cs = (int64_t)Hkv * pre + (int64_t)kvh * nch, ce = cs + nch;
-        const int64_t ps = max(rg.x0, cs), pe = min(rg.x1, ce);
-        const int32_t t_begin = (int32_t)((ps - cs) * kDecChunk);
-        const int32_t t_end = min(ntok, (int32_t)((pe - cs) * kDecChunk));
+        const int32_t cs = Hkv * pre + kvh * nch, ce = cs + nch;
+        const int32_t ps = max(rg.x0, cs), pe = min(rg.x1, ce);
         const bool whole = ps == cs && pe == ce;
-        const int nchunks = (t_end - t_begin + kDmChunk - 1) / kDmChunk;
-
-        // the block ids this piece needs, fetched once (entries t_begin..t_end-1)
         const int32_t *bt = block_table + (int64_t)b * max_blocks;
-        const int32_t blk0 = t_begin / bs;
-        const int32_t nblk = (t_end - 1) / bs - blk0 + 1;
-        // an id outside the pool is reported and kept as -1: its entries are never
-        // copied and count as masked (score -inf, value row zero)
-        for (int i = threadIdx.x; i < nblk; i += blockDim.x) {
-            int32_t id = bt[blk0 + i];
-            if (id < 0 || id >= pool_blocks) {
-                set_status(status, KVS_ERR_INVALID_ARG);
-                id = -1;
-            }
-            S.blk[i] = id;
-        }
-        __syncthreads();
         const int64_t head_off = (int64_t)kvh * bs * D;
-
-        // this warp's chunks are w, w + kDmWarps, ...; each lane copies 16-byte piece
-        // (lane & 15) of entries (lane >> 4) + 2j, j = 0..7, for both K and V
-        auto issue = [&](int i) {
-            const int c = w + i * kDmWarps;
-            if (c < nchunks) {
-                const int s = i % kDmStages;
-                const int32_t t0 = t_begin + c * kDmChunk;
-                const int nv = min(kDmChunk, t_end - t0);
-                const uint32_t kd = smem_u32(S.k[w][s]) + piece * 16, vd = smem_u32(S.v[w][s]) + piece * 16;
-                if constexpr (BS == kDmChunk) {
-                    // pieces start at multiples of 16 entries, so a chunk is exactly one block
-                    const int32_t id = S.blk[t0 / kDmChunk - blk0];
-                    const int64_t base = (int64_t)id * blk_stride + head_off + piece * 8;
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        const int e = par + 2 * j;
-                        if (e < nv && id >= 0) {
-                            cp_async16(kd + e * kDmRow, kc + base + e * D);
-                            cp_async16(vd + e * kDmRow, vc + base + e * D);
-                        }
-                    }
-                } else {
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        const int e = par + 2 * j;
-                        if (e < nv) {
-                            const int32_t t = t0 + e;
-                            const int32_t id = BS == 1 ? S.blk[t - blk0] : S.blk[t / bs - blk0];
-                            const int64_t off = BS == 1 ? (int64_t)id * blk_stride + head_off + piece * 8
-                                                        : (int64_t)id * blk_stride + head_off +
-                                                              (int64_t)(t % bs) * D + piece * 8;
-                            if (id >= 0) {
-                                cp_async16(kd + e * kDmRow, kc + off);
-                                cp_async16(vd + e * kDmRow, vc + off);
-                            }
-                        }
-                    }
-                }
-            }
-            cp_async_commit();  // one group per step, empty past the end
-        };
 
         // Q as the A operand: rows = query heads (rows >= G are zero), 16 dims per k-step
         uint32_t qa[8][4];
@@ -184,104 +124,170 @@ __global__ void __launch_bounds__(kDmThreads, 3)
             qa[kk][2] = g < G ? *reinterpret_cast<const uint32_t *>(qb + g * D + c0 + 8) : 0u;
             qa[kk][3] = g + 8 < G ? *reinterpret_cast<const uint32_t *>(qb + (g + 8) * D + c0 + 8) : 0u;
         }
-#pragma unroll
-        for (int i = 0; i < kDmStages - 1; ++i) issue(i);
-
         float acc[16][4];
 #pragma unroll
         for (int i = 0; i < 16; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
         float mrow = -INFINITY, lrow = 0.f;  // row g (head g); rows g+8 are padding
-        for (int i = 0, c = w; c < nchunks; ++i, c += kDmWarps) {
-            issue(i + kDmStages - 1);
-            cp_async_wait<kDmStages - 1>();  // this lane's copies of chunk i are done
-            __syncwarp();                    // ... and those of the other lanes
-            const int s = i % kDmStages;
-            const int32_t t0 = t_begin + c * kDmChunk;
-            const int nv = min(kDmChunk, t_end - t0);
-            const uint32_t ks = smem_u32(S.k[w][s]), vs = smem_u32(S.v[w][s]);
-            // this lane's entries 2 t4, 2 t4 + 1, 8 + 2 t4, 9 + 2 t4: inside the piece
-            // and with a block id in the pool (the others were not copied)
-            auto entry_ok = [&](int e) -> bool {
-                if (e >= nv) return false;
-                const int32_t t = t0 + e;
-                const int32_t id = BS == kDmChunk ? S.blk[t0 / kDmChunk - blk0]
-                                                  : (BS == 1 ? S.blk[t - blk0] : S.blk[t / bs - blk0]);
-                return id >= 0;
+
+        // sub-pieces of at most kDecMaxChunksPerCta chunks: the table slice of each is
+        // staged in shared memory; the softmax state carries over
+        for (int32_t sp = ps; sp < pe; sp += kDecMaxChunksPerCta) {
+            const int32_t spe = min(pe, sp + kDecMaxChunksPerCta);
+            const int32_t t_begin = (sp - cs) * kDecChunk;
+            const int32_t t_end = min(ntok, (spe - cs) * kDecChunk);
+            const int nchunks = (t_end - t_begin + kDmChunk - 1) / kDmChunk;
+            // the block ids this sub-piece needs (entries t_begin..t_end-1); an id
+            // outside the pool is reported and kept as -1: its entries are never
+            // copied and count as masked (score -inf, value row zero)
+            const int32_t blk0 = t_begin / bs;
+            const int32_t nblk = (t_end - 1) / bs - blk0 + 1;
+            __syncthreads();  // the previous sub-piece is done with the slice and the rings
+            for (int i = threadIdx.x; i < nblk; i += blockDim.x) {
+                int32_t id = bt[blk0 + i];
+                if (id < 0 || id >= pool_blocks) {
+                    set_status(status, KVS_ERR_INVALID_ARG);
+                    id = -1;
+                }
+                S.blk[i] = id;
+            }
+            __syncthreads();
+
+            // this warp's chunks are w, w + kDmWarps, ...; each lane copies 16-byte piece
+            // (lane & 15) of entries (lane >> 4) + 2j, j = 0..7, for both K and V
+            auto issue = [&](int i) {
+                const int c = w + i * kDmWarps;
+                if (c < nchunks) {
+                    const int s = i % kDmStages;
+                    const int32_t t0 = t_begin + c * kDmChunk;
+                    const int nv = min(kDmChunk, t_end - t0);
+                    const uint32_t kd = smem_u32(S.k[w][s]) + piece * 16, vd = smem_u32(S.v[w][s]) + piece * 16;
+                    if constexpr (BS == kDmChunk) {
+                        // sub-pieces start at multiples of 16 entries, so a chunk is exactly one block
+                        const int32_t id = S.blk[t0 / kDmChunk - blk0];
+                        const int64_t base = (int64_t)id * blk_stride + head_off + piece * 8;
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            const int e = par + 2 * j;
+                            if (e < nv && id >= 0) {
+                                cp_async16(kd + e * kDmRow, kc + base + e * D);
+                                cp_async16(vd + e * kDmRow, vc + base + e * D);
+                            }
+                        }
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            const int e = par + 2 * j;
+                            if (e < nv) {
+                                const int32_t t = t0 + e;
+                                const int32_t id = BS == 1 ? S.blk[t - blk0] : S.blk[t / bs - blk0];
+                                const int64_t off = BS == 1 ? (int64_t)id * blk_stride + head_off + piece * 8
+                                                            : (int64_t)id * blk_stride + head_off +
+                                                                  (int64_t)(t % bs) * D + piece * 8;
+                                if (id >= 0) {
+                                    cp_async16(kd + e * kDmRow, kc + off);
+                                    cp_async16(vd + e * kDmRow, vc + off);
+                                }
+                            }
+                        }
+                    }
+                }
+                cp_async_commit();  // one group per step, empty past the end
             };
-            const bool ok0 = entry_ok(2 * t4), ok1 = entry_ok(2 * t4 + 1), ok2 = entry_ok(8 + 2 * t4),
-                       ok3 = entry_ok(9 + 2 * t4);
-            const bool chunk_ok = __all_sync(0xffffffffu, ok0 && ok1 && ok2 && ok3);
-            const bool okv[4] = {ok0, ok1, ok2, ok3};
-            // S = Q K^T for entries 0..7 (j = 0) and 8..15 (j = 1)
-            float sc[2][4];
 #pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                sc[j][0] = sc[j][1] = sc[j][2] = sc[j][3] = 0.f;
+            for (int i = 0; i < kDmStages - 1; ++i) issue(i);
+
+            for (int i = 0, c = w; c < nchunks; ++i, c += kDmWarps) {
+                issue(i + kDmStages - 1);
+                cp_async_wait<kDmStages - 1>();  // this lane's copies of chunk i are done
+                __syncwarp();                    // ... and those of the other lanes
+                const int s = i % kDmStages;
+                const int32_t t0 = t_begin + c * kDmChunk;
+                const int nv = min(kDmChunk, t_end - t0);
+                const uint32_t ks = smem_u32(S.k[w][s]), vs = smem_u32(S.v[w][s]);
+                // this lane's entries 2 t4, 2 t4 + 1, 8 + 2 t4, 9 + 2 t4: inside the piece
+                // and with a block id in the pool (the others were not copied)
+                auto entry_ok = [&](int e) -> bool {
+                    if (e >= nv) return false;
+                    const int32_t t = t0 + e;
+                    const int32_t id = BS == kDmChunk ? S.blk[t0 / kDmChunk - blk0]
+                                                      : (BS == 1 ? S.blk[t - blk0] : S.blk[t / bs - blk0]);
+                    return id >= 0;
+                };
+                const bool ok0 = entry_ok(2 * t4), ok1 = entry_ok(2 * t4 + 1), ok2 = entry_ok(8 + 2 * t4),
+                           ok3 = entry_ok(9 + 2 * t4);
+                const bool chunk_ok = __all_sync(0xffffffffu, ok0 && ok1 && ok2 && ok3);
+                const bool okv[4] = {ok0, ok1, ok2, ok3};
+                // S = Q K^T for entries 0..7 (j = 0) and 8..15 (j = 1)
+                float sc[2][4];
 #pragma unroll
-                for (int kk = 0; kk < 8; kk += 2) {
+                for (int j = 0; j < 2; ++j) {
+                    sc[j][0] = sc[j][1] = sc[j][2] = sc[j][3] = 0.f;
+#pragma unroll
+                    for (int kk = 0; kk < 8; kk += 2) {
+                        uint32_t b0, b1, b2, b3;
+                        const uint32_t addr = ks + (8 * j + (lane & 7)) * kDmRow + kk * 32 + (lane >> 3) * 16;
+                        ldsm_x4(addr, b0, b1, b2, b3);
+                        mma16816(sc[j], qa[kk], b0, b1);
+                        mma16816(sc[j], qa[kk + 1], b2, b3);
+                    }
+                }
+                // online softmax on row g: entries 8j + 2 t4 + {0, 1}
+                float x[4];
+                float cm = -INFINITY;
+#pragma unroll
+                for (int j = 0; j < 2; ++j)
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        x[2 * j + u] = okv[2 * j + u] ? sc[j][u] * scale_log2 : -INFINITY;
+                        cm = fmaxf(cm, x[2 * j + u]);
+                    }
+                cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, 1));
+                cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, 2));
+                const float mn = fmaxf(mrow, cm);
+                const float mref = mn == -INFINITY ? 0.f : mn;
+                const float alpha = ex2(mrow - mref);
+                float p[4], psum = 0.f;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    p[u] = ex2(x[u] - mref);
+                    psum += p[u];
+                }
+                psum += __shfl_xor_sync(0xffffffffu, psum, 1);
+                psum += __shfl_xor_sync(0xffffffffu, psum, 2);
+                lrow = lrow * alpha + psum;
+                mrow = mn;
+                // P as the A operand (rows g, entries 2 t4 (+8)); padding rows stay zero
+                const uint32_t pa[4] = {pack_bf16(p[0], p[1]), 0u, pack_bf16(p[2], p[3]), 0u};
+                // value rows of entries that were not copied this time (past the piece's
+                // end, or with an id outside the pool) hold stale data: zero them
+                const bool z0 = !ok0, z1 = !ok1, z2 = !ok2, z3 = !ok3;
+#pragma unroll
+                for (int dt = 0; dt < 16; dt += 2) {
                     uint32_t b0, b1, b2, b3;
-                    const uint32_t addr = ks + (8 * j + (lane & 7)) * kDmRow + kk * 32 + (lane >> 3) * 16;
-                    ldsm_x4(addr, b0, b1, b2, b3);
-                    mma16816(sc[j], qa[kk], b0, b1);
-                    mma16816(sc[j], qa[kk + 1], b2, b3);
+                    const int row = (lane & 7) + ((lane >> 3) & 1) * 8;
+                    const uint32_t addr = vs + row * kDmRow + (dt + (lane >> 4)) * 16;
+                    ldsm_x4_t(addr, b0, b1, b2, b3);
+                    if (!chunk_ok) {
+                        b0 = (z0 ? b0 & 0xFFFF0000u : b0);
+                        b0 = (z1 ? b0 & 0x0000FFFFu : b0);
+                        b1 = (z2 ? b1 & 0xFFFF0000u : b1);
+                        b1 = (z3 ? b1 & 0x0000FFFFu : b1);
+                        b2 = (z0 ? b2 & 0xFFFF0000u : b2);
+                        b2 = (z1 ? b2 & 0x0000FFFFu : b2);
+                        b3 = (z2 ? b3 & 0xFFFF0000u : b3);
+                        b3 = (z3 ? b3 & 0x0000FFFFu : b3);
+                    }
+                    acc[dt][0] *= alpha;
+                    acc[dt][1] *= alpha;
+                    acc[dt + 1][0] *= alpha;
+                    acc[dt + 1][1] *= alpha;
+                    mma16816(acc[dt], pa, b0, b1);
+                    mma16816(acc[dt + 1], pa, b2, b3);
                 }
+                __syncwarp();  // stage s is refilled by the next iteration's issue
             }
-            // online softmax on row g: entries 8j + 2 t4 + {0, 1}
-            float x[4];
-            float cm = -INFINITY;
-#pragma unroll
-            for (int j = 0; j < 2; ++j)
-#pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    x[2 * j + u] = okv[2 * j + u] ? sc[j][u] * scale_log2 : -INFINITY;
-                    cm = fmaxf(cm, x[2 * j + u]);
-                }
-            cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, 1));
-            cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, 2));
-            const float mn = fmaxf(mrow, cm);
-            const float mref = mn == -INFINITY ? 0.f : mn;
-            const float alpha = ex2(mrow - mref);
-            float p[4], psum = 0.f;
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                p[u] = ex2(x[u] - mref);
-                psum += p[u];
-            }
-            psum += __shfl_xor_sync(0xffffffffu, psum, 1);
-            psum += __shfl_xor_sync(0xffffffffu, psum, 2);
-            lrow = lrow * alpha + psum;
-            mrow = mn;
-            // P as the A operand (rows g, entries 2 t4 (+8)); padding rows stay zero
-            const uint32_t pa[4] = {pack_bf16(p[0], p[1]), 0u, pack_bf16(p[2], p[3]), 0u};
-            // value rows of entries that were not copied this time (past the piece's
-            // end, or with an id outside the pool) hold stale data: zero them
-            const bool z0 = !ok0, z1 = !ok1, z2 = !ok2, z3 = !ok3;
-#pragma unroll
-            for (int dt = 0; dt < 16; dt += 2) {
-                uint32_t b0, b1, b2, b3;
-                const int row = (lane & 7) + ((lane >> 3) & 1) * 8;
-                const uint32_t addr = vs + row * kDmRow + (dt + (lane >> 4)) * 16;
-                ldsm_x4_t(addr, b0, b1, b2, b3);
-                if (!chunk_ok) {
-                    b0 = (z0 ? b0 & 0xFFFF0000u : b0);
-                    b0 = (z1 ? b0 & 0x0000FFFFu : b0);
-                    b1 = (z2 ? b1 & 0xFFFF0000u : b1);
-                    b1 = (z3 ? b1 & 0x0000FFFFu : b1);
-                    b2 = (z0 ? b2 & 0xFFFF0000u : b2);
-                    b2 = (z1 ? b2 & 0x0000FFFFu : b2);
-                    b3 = (z2 ? b3 & 0xFFFF0000u : b3);
-                    b3 = (z3 ? b3 & 0x0000FFFFu : b3);
-                }
-                acc[dt][0] *= alpha;
-                acc[dt][1] *= alpha;
-                acc[dt + 1][0] *= alpha;
-                acc[dt + 1][1] *= alpha;
-                mma16816(acc[dt], pa, b0, b1);
-                mma16816(acc[dt + 1], pa, b2, b3);
-            }
-            __syncwarp();  // stage s is refilled by the next iteration's issue
+            cp_async_wait<0>();
         }
-        cp_async_wait<0>();
         if (t4 == 0 && g < G) {
             S.m[w][g] = mrow;
             S.l[w][g] = lrow;
@@ -326,7 +332,7 @@ __global__ void __launch_bounds__(kDmThreads, 3)
             }
         }
         if (pe >= rg.x1) break;
-        __syncthreads();  // the next piece refills the rings and the table slice
+        __syncthreads();  // the next piece refills the rings (which hold cacc) and the slice
         // next unit: the next kv head, or the next sequence with live entries
         if (++kvh == Hkv) {
             kvh = 0;

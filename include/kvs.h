@@ -192,13 +192,13 @@ kvs_status kvs_rope_logical(const void *x, int64_t x_tok_stride, void *y, const 
  *   ws      device scratch of kvs_paged_decode_ws_bytes(...) bytes; no
  *           initialisation needed. Work split: the live entries of unit
  *           (b, kv head) are cut into chunks of 16; the units' chunks are laid
- *           end to end and C CTAs take equal consecutive shares of them
- *           (C = ceil(B*Hkv*ceil(max_blocks*block_size/16) / 72), rounded up to
- *           a multiple of 444 = 148 SMs x 3, at most the chunk count), so the
- *           split follows the actual num_tokens, found on the device. Scratch =
- *           8*(B+1) bytes of prefix counts (rounded up to 256) + (C + B*Hkv)
- *           partial results of G*(d+2) fp32. The call runs the split kernel
- *           and a merge kernel.
+ *           end to end and C = min(444, B*Hkv*ceil(max_blocks*block_size/16))
+ *           CTAs (one wave of 148 SMs x 3) take equal consecutive shares of
+ *           them, found on the device from num_tokens. Scratch = 8*(B+1) bytes
+ *           of prefix counts (rounded up to 256) + (C + B*Hkv) partial results
+ *           of G*(d+2) fp32. The call runs the split kernel and a merge kernel.
+ *           The table's chunk count B*Hkv*ceil(max_blocks*block_size/16) must
+ *           fit in int32 (else KVS_ERR_CAPACITY).
  * Errors found in device data set KVS_ERR_INVALID_ARG in *dev_status:
  *  - a block id outside [0, pool_blocks): none of its entries is read; they
  *    are left out of the softmax (as if evicted);

@@ -74,15 +74,11 @@ def test_product_path_has_no_oracle_import():
 
 
 def _plan_ws(B, Hq, Hkv, d, bs, max_blocks):
-    """The work split as documented at kvs_paged_decode_ws_bytes: C CTAs, enough that
-    none takes more than 72 chunks of 16 entries when every table is full, rounded up to
-    whole waves of 444 (and no more than the chunks); scratch = 8 (B + 1) bytes of
-    prefix counts (rounded up to 256) + (C + B Hkv) G (d + 2) fp32 partials."""
-    mc = -(-(max_blocks * bs) // 16)
-    tc = B * Hkv * mc
-    c = -(-tc // 72)
-    c = -(-c // 444) * 444
-    c = max(1, min(c, tc))
+    """The work split as documented at kvs_paged_decode_ws_bytes: C = min(444, chunks of
+    the full table) CTAs; scratch = 8 (B + 1) bytes of prefix counts (rounded up to 256)
+    + (C + B Hkv) G (d + 2) fp32 partials."""
+    tc = B * Hkv * -(-(max_blocks * bs) // 16)
+    c = max(1, min(444, tc))
     G = Hq // Hkv
     return -(-(8 * (B + 1)) // 256) * 256 + (c + B * Hkv) * G * (d + 2) * 4
 

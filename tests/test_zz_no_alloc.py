@@ -62,7 +62,7 @@ def test_static_decode_matches_regular_entry_point(bs):
 
 
 def test_static_decode_rejects_oversized_requests():
-    B, Hq, Hkv, d, bs, M = 64, 32, 8, 128, 16, 2049
+    B, Hq, Hkv, d, bs, M = 4096, 64, 8, 128, 16, 64
     assert kvs.lib().kvs_paged_decode_ws_bytes(B, Hq, Hkv, d, bs, M) > STATIC_MAX
     t = torch.zeros(1, dtype=torch.bfloat16, device="cuda")
     i = torch.zeros(1, dtype=torch.int32, device="cuda")
