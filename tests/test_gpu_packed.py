@@ -12,8 +12,7 @@ import oracle
 import eviction_masked_attention_b200 as kvs
 from eviction_masked_attention_b200 import packing
 from eviction_masked_attention_b200 import workloads as W
-from gpu_util import (BF16_TOL, F32_ROUND, F32_TOL, GRAD_REL_L2, LSE_TOL, assert_close, dev, events_dev,
-                      host, rel_l2)
+from gpu_util import BF16_TOL, F32_ROUND, F32_TOL, GRAD_REL_L2, assert_close, dev, events_dev, host, rel_l2
 
 pytestmark = pytest.mark.gpu
 
@@ -57,7 +56,10 @@ def test_packed_policy_mix_fwd_bwd(dtype):
                                                 kap, scale)
         name = mix[b].name
         assert_close(host(o[0, sl]), wo[0], tol, f"O packed {name}")
-        assert_close(host(lse[0][:, sl]), wl[0], LSE_TOL if dtype == "bf16" else F32_TOL, f"LSE packed {name}",
+        # the attention inputs here are the rotary kernel's bf16 outputs: their rounding
+        # (2^-9 per element) moves a score by up to ~2^-8 |q||k| scale, which the
+        # exact-input log-sum-exp bound does not cover; bf16 inputs get the bf16 bound
+        assert_close(host(lse[0][:, sl]), wl[0], BF16_TOL if dtype == "bf16" else F32_TOL, f"LSE packed {name}",
                      rnd=F32_ROUND)
         for nm, got, want in (("dq", dq, wdq), ("dk", dk, wdk), ("dv", dv, wdv)):
             g_ = host(got[0, sl])
