@@ -106,21 +106,30 @@ __device__ __forceinline__ void store_row64(__nv_bfloat16 *dst, const uint32_t (
 // they had read it.
 
 constexpr int kBwdThreads = 320;  // warp 0 TMA, warp 1 MMA, warps 2..9 elementwise
-constexpr int kDkvStages = 2;
+// Q(n) is read by S^T(n) and dK(n), dO(n) by dP^T(n) and dV(n). With three Q
+// stages the load of Q(n+3) goes out when dK(n) completes, six products before
+// S^T(n+3); with two dO stages the load of dO(n+2) goes out when dV(n)
+// completes, six products before dP^T(n+2). The rows' -LSE log2(e) and D (and
+// the tile's origin and class) ride on a 2-stage ring of their own that the
+// elementwise warps release when they finish an item.
+constexpr int kDkvQStages = 3, kDkvOStages = 2, kDkvRowStages = 2;
 
 struct DkvSmem {
     uint8_t k[kTile];
     uint8_t v[kTile];
-    uint8_t q[kDkvStages][kTile];
-    uint8_t dout[kDkvStages][kTile];
-    float nl2[kDkvStages][128];  // -lse log2(e) of the tile's rows
-    float dd[kDkvStages][128];
-    int32_t q0[kDkvStages], full_tile[kDkvStages];  // tile origin, FULL flag
-    uint64_t kv_full, full[kDkvStages], empty[kDkvStages], st_full, dp_full, p_ready, ds_ready,
-        acc_done, fin;
+    uint8_t q[kDkvQStages][kTile];
+    uint8_t dout[kDkvOStages][kTile];
+    float nl2[kDkvRowStages][128];  // -lse log2(e) of the tile's rows
+    float dd[kDkvRowStages][128];
+    int32_t q0[kDkvRowStages], full_tile[kDkvRowStages];  // tile origin, FULL flag
+    uint64_t kv_full, qfull[kDkvQStages], qempty[kDkvQStages], ofull[kDkvOStages], oempty[kDkvOStages],
+        rfull[kDkvRowStages], rempty[kDkvRowStages], st_full, dp_full, p_ready, ds_ready, acc_done, fin;
     uint32_t tmem_base;
     int abort;
 };
+// the whole budget of dynamic shared memory; the kernel checks that its base is
+// 1024-byte aligned (the swizzled tiles need it) instead of padding for it
+static_assert(sizeof(DkvSmem) <= 232448, "dK/dV shared memory over the 227 KB limit");
 
 // TMEM column of the bf16 pairs of rows 16kk..16kk+15 inside a 128-column region
 // whose halves hold rows 0..63 and 64..127 in their first 32 columns.
@@ -132,9 +141,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                    kvs_tile_mask m, int32_t Hq, int32_t Hkv, float scale, float scale_log2,
                    const float *__restrict__ Drow, const float *__restrict__ NL2,
                    __nv_bfloat16 *__restrict__ dk, __nv_bfloat16 *__restrict__ dv, int32_t *status) {
-    extern __shared__ uint8_t smem_raw[];
-    DkvSmem &S = *reinterpret_cast<DkvSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    DkvSmem &S = *reinterpret_cast<DkvSmem *>(smem_raw);
+    if (smem_u32(smem_raw) & 1023u) {  // same for every thread of the CTA
+        if (threadIdx.x == 0) set_status(status, KVS_ERR_UNSUPPORTED);
+        return;
+    }
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int B = m.B, N = m.N, T = m.T, G = Hq / Hkv, Tpad = T * 128;
     // key tiles with the longest column lists (small kj) first
@@ -149,9 +161,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
     if (threadIdx.x == 0) {
         mbar_init(&S.kv_full, 1);
-        for (int i = 0; i < kDkvStages; ++i) {
-            mbar_init(&S.full[i], 1);
-            mbar_init(&S.empty[i], 1);
+        for (int i = 0; i < kDkvQStages; ++i) {
+            mbar_init(&S.qfull[i], 1);
+            mbar_init(&S.qempty[i], 1);
+        }
+        for (int i = 0; i < kDkvOStages; ++i) {
+            mbar_init(&S.ofull[i], 1);
+            mbar_init(&S.oempty[i], 1);
+        }
+        for (int i = 0; i < kDkvRowStages; ++i) {
+            mbar_init(&S.rfull[i], 1);
+            mbar_init(&S.rempty[i], 256);
         }
         mbar_init(&S.st_full, 1);
         mbar_init(&S.dp_full, 1);
@@ -180,23 +200,40 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             tma_load_4d(S.k + kTile / 2, &tmK, &S.kv_full, 64, kvh, k0, b);
             tma_load_4d(S.v, &tmV, &S.kv_full, 0, kvh, k0, b);
             tma_load_4d(S.v + kTile / 2, &tmV, &S.kv_full, 64, kvh, k0, b);
+            // Q(n) once dK(n-3) is done, dO(n) once dV(n-2) is done
             for (int n = 0; n < nw; ++n) {
-                const int s = n % kDkvStages;
-                if (n >= kDkvStages &&
-                    !mbar_wait(&S.empty[s], ((n / kDkvStages) - 1) & 1, abort, status))
-                    break;
                 const int e = n / G, h = kvh * G + n % G;
                 const int q0 = m.col_row[c0 + e] * 128;
-                S.q0[s] = q0;
-                S.full_tile[s] = m.col_pidx[c0 + e] < 0;
-                mbar_expect_tx(&S.full[s], 2 * kTile + 1024);
-                tma_load_4d(S.q[s], &tmQ, &S.full[s], 0, h, q0, b);
-                tma_load_4d(S.q[s] + kTile / 2, &tmQ, &S.full[s], 64, h, q0, b);
-                tma_load_4d(S.dout[s], &tmO, &S.full[s], 0, h, q0, b);
-                tma_load_4d(S.dout[s] + kTile / 2, &tmO, &S.full[s], 64, h, q0, b);
+                const int qs = n % kDkvQStages;
+                if (n >= kDkvQStages &&
+                    !mbar_wait(&S.qempty[qs], ((n / kDkvQStages) - 1) & 1, abort, status))
+                    break;
+                mbar_expect_tx(&S.qfull[qs], kTile);
+                tma_load_4d(S.q[qs], &tmQ, &S.qfull[qs], 0, h, q0, b);
+                tma_load_4d(S.q[qs] + kTile / 2, &tmQ, &S.qfull[qs], 64, h, q0, b);
+                const int os = n % kDkvOStages;
+                if (n >= kDkvOStages &&
+                    !mbar_wait(&S.oempty[os], ((n / kDkvOStages) - 1) & 1, abort, status))
+                    break;
+                mbar_expect_tx(&S.ofull[os], kTile);
+                tma_load_4d(S.dout[os], &tmO, &S.ofull[os], 0, h, q0, b);
+                tma_load_4d(S.dout[os] + kTile / 2, &tmO, &S.ofull[os], 64, h, q0, b);
+            }
+        } else if (lane == 1 && nw > 0) {
+            // the items' row data, each once the elementwise warps are done with item n-2
+            for (int n = 0; n < nw; ++n) {
+                const int e = n / G, h = kvh * G + n % G;
+                const int q0 = m.col_row[c0 + e] * 128;
                 const int64_t ro = ((int64_t)b * Hq + h) * Tpad + q0;
-                bulk_load(S.nl2[s], NL2 + ro, 512, &S.full[s]);
-                bulk_load(S.dd[s], Drow + ro, 512, &S.full[s]);
+                const int rs = n % kDkvRowStages;
+                if (n >= kDkvRowStages &&
+                    !mbar_wait(&S.rempty[rs], ((n / kDkvRowStages) - 1) & 1, abort, status))
+                    break;
+                S.q0[rs] = q0;
+                S.full_tile[rs] = m.col_pidx[c0 + e] < 0;
+                mbar_expect_tx(&S.rfull[rs], 1024);
+                bulk_load(S.nl2[rs], NL2 + ro, 512, &S.rfull[rs]);
+                bulk_load(S.dd[rs], Drow + ro, 512, &S.rfull[rs]);
             }
         }
     } else if (warp == 1) {
@@ -211,25 +248,37 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             const uint64_t ok0 = sw128_desc(smem_u32(S.dout[0]), 16, 1024);
             const uint64_t qm0 = sw128_desc(smem_u32(S.q[0]), kTile / 2, 1024);
             const uint64_t om0 = sw128_desc(smem_u32(S.dout[0]), kTile / 2, 1024);
-            // S^T = K Q^T and dP^T = V dO^T of item n (its stage already waited for)
-            auto issue_t = [&](int n, uint64_t a, uint64_t b0, uint32_t dst, uint64_t *bar) {
-                const uint64_t bd = desc_add(b0, (n % kDkvStages) * kTile);  // q[s], dout[s]: kTile apart
+            // S^T(n) = K Q(n)^T and dP^T(n) = V dO(n)^T
+            auto issue_st = [&](int n) -> bool {
+                const int qs = n % kDkvQStages;
+                if (!warp_wait(&S.qfull[qs], (n / kDkvQStages) & 1, abort, status)) return false;
+                tc_fence_after();
+                const uint64_t bd = desc_add(qk0, qs * kTile);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint32_t off = (kk >> 2) * (kTile / 2) + (kk & 3) * 32;
-                    if (leader) mma_ss(dst, desc_add(a, off), desc_add(bd, off), idT, kk > 0);
+                    if (leader) mma_ss(tmem + cST, desc_add(kd, off), desc_add(bd, off), idT, kk > 0);
                 }
-                if (leader) mma_commit(bar);
+                if (leader) mma_commit(&S.st_full);
+                return true;
             };
-            bool ok = warp_wait(&S.kv_full, 0, abort, status) && warp_wait(&S.full[0], 0, abort, status);
-            if (ok) {
+            auto issue_dp = [&](int n) -> bool {
+                const int os = n % kDkvOStages;
+                if (!warp_wait(&S.ofull[os], (n / kDkvOStages) & 1, abort, status)) return false;
                 tc_fence_after();
-                issue_t(0, kd, qk0, tmem + cST, &S.st_full);
-                issue_t(0, vd, ok0, tmem + cDP, &S.dp_full);
-            }
+                const uint64_t bd = desc_add(ok0, os * kTile);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t off = (kk >> 2) * (kTile / 2) + (kk & 3) * 32;
+                    if (leader) mma_ss(tmem + cDP, desc_add(vd, off), desc_add(bd, off), idT, kk > 0);
+                }
+                if (leader) mma_commit(&S.dp_full);
+                return true;
+            };
+            bool ok = warp_wait(&S.kv_full, 0, abort, status) && issue_st(0) && issue_dp(0);
             for (int n = 0; ok && n < nw; ++n) {
-                const int s = n % kDkvStages;
-                const uint64_t qm = desc_add(qm0, s * kTile), om = desc_add(om0, s * kTile);
+                const uint64_t qm = desc_add(qm0, (n % kDkvQStages) * kTile);
+                const uint64_t om = desc_add(om0, (n % kDkvOStages) * kTile);
                 const uint32_t acc = n > 0 ? 1u : 0u;
                 if (!warp_wait(&S.p_ready, n & 1, abort, status)) break;
                 tc_fence_after();
@@ -238,13 +287,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     if (leader)
                         mma_ts(tmem + cDV, tmem + cST + packed_col(kk), desc_add(om, kk * 2048), idMN,
                                kk > 0 ? 1u : acc);
+                if (leader) mma_commit(&S.oempty[n % kDkvOStages]);
                 const bool more = n + 1 < nw;
-                if (more) {
-                    if (!warp_wait(&S.full[(n + 1) % kDkvStages], ((n + 1) / kDkvStages) & 1, abort, status))
-                        break;
-                    tc_fence_after();
-                    issue_t(n + 1, kd, qk0, tmem + cST, &S.st_full);
-                }
+                if (more && !issue_st(n + 1)) break;
                 if (!warp_wait(&S.ds_ready, n & 1, abort, status)) break;
                 tc_fence_after();
 #pragma unroll
@@ -252,8 +297,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     if (leader)
                         mma_ts(tmem + cDK, tmem + cDP + packed_col(kk), desc_add(qm, kk * 2048), idMN,
                                kk > 0 ? 1u : acc);
-                if (leader) mma_commit(&S.empty[s]);
-                if (more) issue_t(n + 1, vd, ok0, tmem + cDP, &S.dp_full);
+                if (leader) mma_commit(&S.qempty[n % kDkvQStages]);
+                if (more && !issue_dp(n + 1)) break;
             }
             if (leader) mma_commit(&S.acc_done);
             if (leader) mma_commit(&S.fin);
@@ -269,9 +314,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const int32_t kap = j < N ? m.kappa[(int64_t)b * N + j] : 0;
         bool ok = true;
         for (int n = 0; n < nw; ++n) {
-            const int s = n % kDkvStages;
+            const int s = n % kDkvRowStages;
             const uint32_t ph = n & 1;
-            if (!warp_wait(&S.full[s], (n / kDkvStages) & 1, abort, status)) {
+            if (!warp_wait(&S.rfull[s], (n / kDkvRowStages) & 1, abort, status)) {
                 ok = false;
                 break;
             }
@@ -373,6 +418,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             tmem_st_wait();
             tc_fence_before();
             mbar_arrive(&S.ds_ready);
+            mbar_arrive(&S.rempty[s]);  // done with this item's row data
         }
         // each group writes 64 of the 128 dimensions of dV and dK
         const uint32_t col0 = h * 64;
@@ -405,36 +451,37 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
 // ---------------------------------------------------------------------- dQ
 //
-// TMEM: S [0,128), dP [128,256), dQ accumulator [256,384), dS double buffer
-// [384,448) [448,512) (bf16 pairs). Because dS has its own buffers, S and dP of
-// the next key tile are issued as soon as the elementwise warps have read the
-// current ones, so the tensor core computes them while dS is being formed.
-
-// K is needed from S_n until dQ_n, at the end of the item, V only for dP_n. K
-// has three stages, so the load of K_{n+1} goes out when dQ_{n-2} completes,
-// an item ahead of S_{n+1}; V has two, so V_{n+1} goes out when dP_{n-1}
-// completes, four products ahead of dP_{n+1}. (With one V stage the load of
-// V_{n+1} waited for dP_n, only S_{n+1} ahead of its use.) The mask rows of a
-// partial tile are read by each elementwise thread from global memory (L2)
-// while it waits for S_n: there is no shared memory left for them.
+// TMEM: S [0,128), dP [128,256), dQ accumulator [256,384), and the CTA's Q
+// [384,448) and dO [448,512) as bf16 pairs: S = Q K^T and dP = dO V^T take
+// their A operand from TMEM, so each product reads only K or V from shared
+// memory (160 KB of shared-memory reads and fills per item instead of 224 KB,
+// below the 1536 cycles of tensor work). The eight elementwise warps split an
+// item's 128 keys in two halves (thread = query row); each writes its dS as
+// bf16 pairs into the first 32 of its own 64 columns of dP, the A operand of
+// dQ += dS K. Per item the tensor core runs, in issue order, dP(n),
+// [S(n) read] S(n+1), [dS(n) written] dQ(n), then dP(n+1): each product that
+// overwrites a TMEM region comes after the one that reads it.
+//
+// K is needed from S_n until dQ_n, V only for dP_n. K has three stages (the
+// load of K_{n+2} goes out when dQ_{n-1} completes, 2048 cycles of tensor work
+// before S_{n+2}), V two (V_{n+2} when dP_n completes, five products ahead).
 constexpr int kDqKStages = 3;
 constexpr int kDqVStages = 2;
 
 struct DqSmem {
-    uint8_t q[kTile];
-    uint8_t dout[kTile];
     uint8_t k[kDqKStages][kTile];
     uint8_t v[kDqVStages][kTile];
-    int32_t pid[kDqKStages];  // partial index of the key tile in each K stage (-1: full)
-    uint64_t qo_full, kfull[kDqKStages], kempty[kDqKStages], vfull[kDqVStages], vempty[kDqVStages], s_full,
-        dp_full, s_free, dp_free, ds_ready, dq_done, acc_done, fin;
+    uint32_t bits[kDqKStages][128 * 4];  // mask rows of the key tile in each K stage (partial tiles)
+    int32_t pid[kDqKStages];             // its partial index (-1: full)
+    uint64_t kfull[kDqKStages], kempty[kDqKStages], vfull[kDqVStages], vempty[kDqVStages], qo_ready,
+        s_full, dp_full, s_free, ds_ready, acc_done, fin;
     uint32_t tmem_base;
     int abort;
 };
 
 __global__ void __launch_bounds__(kBwdThreads, 1)
-    k_attn_dq_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+    k_attn_dq_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                 const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ dO,
                  kvs_tile_mask m, int32_t Hq, int32_t Hkv, float scale, float scale_log2,
                  const float *__restrict__ Drow, const float *__restrict__ NL2,
                  __nv_bfloat16 *__restrict__ dq, int32_t *status) {
@@ -452,7 +499,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     if (grid_timed_out(status)) return;
 
     if (threadIdx.x == 0) {
-        mbar_init(&S.qo_full, 1);
         for (int i = 0; i < kDqKStages; ++i) {
             mbar_init(&S.kfull[i], 1);
             mbar_init(&S.kempty[i], 1);
@@ -461,12 +507,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             mbar_init(&S.vfull[i], 1);
             mbar_init(&S.vempty[i], 1);
         }
+        mbar_init(&S.qo_ready, 256);
         mbar_init(&S.s_full, 1);
         mbar_init(&S.dp_full, 1);
         mbar_init(&S.s_free, 256);
-        mbar_init(&S.dp_free, 256);
         mbar_init(&S.ds_ready, 256);
-        mbar_init(&S.dq_done, 1);
         mbar_init(&S.acc_done, 1);
         mbar_init(&S.fin, 1);
         S.abort = 0;
@@ -481,25 +526,22 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     tc_fence_after();
     const uint32_t tmem = S.tmem_base;
     volatile int *abort = &S.abort;
-    constexpr uint32_t cS = 0, cDP = 128, cDQ = 256, cDS = 384;
+    constexpr uint32_t cS = 0, cDP = 128, cDQ = 256, cQ = 384, cO = 448;
 
     if (warp == 0) {
         if (lane == 0 && nt > 0) {
-            mbar_expect_tx(&S.qo_full, 2 * kTile);
-            tma_load_4d(S.q, &tmQ, &S.qo_full, 0, hq, q0, b);
-            tma_load_4d(S.q + kTile / 2, &tmQ, &S.qo_full, 64, hq, q0, b);
-            tma_load_4d(S.dout, &tmO, &S.qo_full, 0, hq, q0, b);
-            tma_load_4d(S.dout + kTile / 2, &tmO, &S.qo_full, 64, hq, q0, b);
             for (int n = 0; n < nt; ++n) {
                 const int ks = n % kDqKStages;
                 const int k0 = m.row_col[e0 + n] * 128;
                 if (n >= kDqKStages &&
                     !mbar_wait(&S.kempty[ks], ((n / kDqKStages) - 1) & 1, abort, status))
                     break;
-                S.pid[ks] = m.row_pidx[e0 + n];
-                mbar_expect_tx(&S.kfull[ks], kTile);
+                const int32_t pid = m.row_pidx[e0 + n];
+                S.pid[ks] = pid;
+                mbar_expect_tx(&S.kfull[ks], kTile + (pid >= 0 ? 2048u : 0u));
                 tma_load_4d(S.k[ks], &tmK, &S.kfull[ks], 0, kvh, k0, b);
                 tma_load_4d(S.k[ks] + kTile / 2, &tmK, &S.kfull[ks], 64, kvh, k0, b);
+                if (pid >= 0) bulk_load(S.bits[ks], m.bits + (int64_t)pid * 512, 2048, &S.kfull[ks]);
                 const int vs = n % kDqVStages;
                 if (n >= kDqVStages &&
                     !mbar_wait(&S.vempty[vs], ((n / kDqVStages) - 1) & 1, abort, status))
@@ -514,24 +556,25 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             const bool leader = elect_one();
             const uint32_t idKM = idesc_bf16(128, 128, false, false);
             const uint32_t idMN = idesc_bf16(128, 128, false, true);
-            const uint64_t qd = sw128_desc(smem_u32(S.q), 16, 1024);
-            const uint64_t od = sw128_desc(smem_u32(S.dout), 16, 1024);
             const uint64_t kd0 = sw128_desc(smem_u32(S.k[0]), 16, 1024);         // + stage * kTile
             const uint64_t km0 = sw128_desc(smem_u32(S.k[0]), kTile / 2, 1024);  // MN-major view
-            const uint64_t vd0 = sw128_desc(smem_u32(S.v[0]), 16, 1024);  // + stage * kTile
-            auto issue_s_dp = [&](int n) -> bool {
+            const uint64_t vd0 = sw128_desc(smem_u32(S.v[0]), 16, 1024);         // + stage * kTile
+            // S(n) = Q K(n)^T, A = Q from TMEM (d in bf16 pairs: K step kk at column 8 kk)
+            auto issue_s = [&](int n) -> bool {
                 const int ks = n % kDqKStages;
                 if (!warp_wait(&S.kfull[ks], (n / kDqKStages) & 1, abort, status)) return false;
-                const uint64_t kd = desc_add(kd0, ks * kTile);
-                if (n > 0 && !warp_wait(&S.s_free, (n - 1) & 1, abort, status)) return false;
                 tc_fence_after();
+                const uint64_t kd = desc_add(kd0, ks * kTile);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint32_t off = (kk >> 2) * (kTile / 2) + (kk & 3) * 32;
-                    if (leader) mma_ss(tmem + cS, desc_add(qd, off), desc_add(kd, off), idKM, kk > 0);
+                    if (leader) mma_ts(tmem + cS, tmem + cQ + 8 * kk, desc_add(kd, off), idKM, kk > 0);
                 }
                 if (leader) mma_commit(&S.s_full);
-                if (n > 0 && !warp_wait(&S.dp_free, (n - 1) & 1, abort, status)) return false;
+                return true;
+            };
+            // dP(n) = dO V(n)^T, A = dO from TMEM
+            auto issue_dp = [&](int n) -> bool {
                 const int vs = n % kDqVStages;
                 if (!warp_wait(&S.vfull[vs], (n / kDqVStages) & 1, abort, status)) return false;
                 tc_fence_after();
@@ -539,25 +582,37 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint32_t off = (kk >> 2) * (kTile / 2) + (kk & 3) * 32;
-                    if (leader) mma_ss(tmem + cDP, desc_add(od, off), desc_add(vd, off), idKM, kk > 0);
+                    if (leader) mma_ts(tmem + cDP, tmem + cO + 8 * kk, desc_add(vd, off), idKM, kk > 0);
                 }
                 if (leader) mma_commit(&S.dp_full);
                 if (leader) mma_commit(&S.vempty[vs]);
                 return true;
             };
-            bool ok = warp_wait(&S.qo_full, 0, abort, status) && issue_s_dp(0);
+            bool ok = warp_wait(&S.qo_ready, 0, abort, status);
+            if (ok) {
+                tc_fence_after();
+                ok = issue_s(0) && issue_dp(0);
+            }
             for (int n = 0; ok && n < nt; ++n) {
-                const int s = n & 1;
-                if (n + 1 < nt && !issue_s_dp(n + 1)) break;
+                const bool more = n + 1 < nt;
+                // S(n+1) overwrites S(n) once the elementwise warps have read it
+                if (more) {
+                    if (!warp_wait(&S.s_free, n & 1, abort, status)) break;
+                    if (!issue_s(n + 1)) break;
+                }
+                // dQ(n) += dS(n) K(n), dS in the dP columns
                 if (!warp_wait(&S.ds_ready, n & 1, abort, status)) break;
                 tc_fence_after();
                 const uint64_t km = desc_add(km0, (n % kDqKStages) * kTile);
-                const uint32_t sa = tmem + cDS + s * 64, acc = n > 0 ? 1u : 0u;
+                const uint32_t acc = n > 0 ? 1u : 0u;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    if (leader) mma_ts(tmem + cDQ, sa + kk * 8, desc_add(km, kk * 2048), idMN, kk > 0 ? 1u : acc);
+                    if (leader)
+                        mma_ts(tmem + cDQ, tmem + cDP + packed_col(kk), desc_add(km, kk * 2048), idMN,
+                               kk > 0 ? 1u : acc);
                 if (leader) mma_commit(&S.kempty[n % kDqKStages]);
-                if (leader) mma_commit(&S.dq_done);
+                // dP(n+1) overwrites dS(n) after dQ(n) has read it (in issue order)
+                if (more && !issue_dp(n + 1)) break;
             }
             if (leader) mma_commit(&S.acc_done);
             if (leader) mma_commit(&S.fin);
@@ -574,20 +629,38 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const float nl2 = NL2[ro], dd = Drow[ro];
         const uint64_t dd2 = f2_make(dd, dd);
         bool ok = true;
+        if (nt > 0) {
+            // this row's half of Q and of dO into TMEM as bf16 pairs (the A operands);
+            // rows past N are zero
+            uint32_t r[32];
+#pragma unroll
+            for (int w = 0; w < 2; ++w) {
+                const __nv_bfloat16 *src = (w ? dO : q) + (((int64_t)b * N + t) * Hq + hq) * 128 + half * 64;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const uint4 u = t < N ? *reinterpret_cast<const uint4 *>(src + 8 * i) : make_uint4(0, 0, 0, 0);
+                    r[4 * i] = u.x;
+                    r[4 * i + 1] = u.y;
+                    r[4 * i + 2] = u.z;
+                    r[4 * i + 3] = u.w;
+                }
+                tmem_st32(tmem + lane_off + (w ? cO : cQ) + half * 32, r);
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(&S.qo_ready);
+        }
         for (int n = 0; n < nt; ++n) {
-            const int s = n & 1;
-            // the K stage carries the tile's partial index; it is refilled only after
-            // dQ_n, i.e. after this item's dS. The mask row comes from global memory,
-            // requested before the wait for S_n.
+            // the K stage carries the tile's mask rows; it is refilled only after
+            // dQ_n, i.e. after this item's dS
             const int ks = n % kDqKStages;
             if (!warp_wait(&S.kfull[ks], (n / kDqKStages) & 1, abort, status)) {
                 ok = false;
                 break;
             }
-            const int32_t pid = S.pid[ks];
-            const bool partial = pid >= 0;  // same for the whole CTA
+            const bool partial = S.pid[ks] >= 0;  // same for the whole CTA
             uint2 bits = make_uint2(~0u, ~0u);
-            if (partial) bits = *reinterpret_cast<const uint2 *>(m.bits + (int64_t)pid * 512 + row * 4 + half * 2);
+            if (partial) bits = *reinterpret_cast<const uint2 *>(&S.bits[ks][row * 4 + half * 2]);
             if (!warp_wait(&S.s_full, n & 1, abort, status)) {
                 ok = false;
                 break;
@@ -634,14 +707,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 break;
             }
             tc_fence_after();
-            uint32_t pk[32];
             {
-                uint32_t r0[32], r1[32];
+                uint32_t r0[32], r1[32], pk[32];
                 tmem_ld32(tmem + lane_off + cDP + col0, r0);
                 tmem_ld32(tmem + lane_off + cDP + col0 + 32, r1);
                 tmem_ld_wait();
-                tc_fence_before();
-                mbar_arrive(&S.dp_free);
 #pragma unroll
                 for (int jj = 0; jj < 32; jj += 2) {
                     float d0, d1, d2, d3;
@@ -655,16 +725,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     pk[jj >> 1] = pack_bf16(d0, d1);
                     pk[16 + (jj >> 1)] = pack_bf16(d2, d3);
                 }
+                // keys col0..col0+63 as bf16 pairs in the first 32 columns of this half
+                tmem_st32(tmem + lane_off + cDP + col0, pk);
             }
-            // dQ of item n-1 must be complete: its MMA has then consumed ds_ready
-            // phase n-1 (so this arrival cannot run two phases ahead) and the
-            // dS buffer written two items ago is free.
-            if (n >= 1 && !warp_wait(&S.dq_done, (n - 1) & 1, abort, status)) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
-            tmem_st32(tmem + lane_off + cDS + s * 64 + half * 32, pk);
             tmem_st_wait();
             tc_fence_before();
             mbar_arrive(&S.ds_ready);
@@ -708,7 +771,7 @@ cudaError_t launch_bwd_tc(const void *q, const void *k, const void *v, const voi
     const float sl2 = scale * 1.4426950408889634f;
     cudaError_t e = cudaSuccess;
     if (stages & KVS_BWD_DKDV) {
-        const size_t smem = sizeof(DkvSmem) + 1024;
+        const size_t smem = sizeof(DkvSmem);
         e = cudaFuncSetAttribute(k_attn_dkdv_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)smem);
         if (e != cudaSuccess) return e;
@@ -722,7 +785,8 @@ cudaError_t launch_bwd_tc(const void *q, const void *k, const void *v, const voi
                                  (int)smem);
         if (e != cudaSuccess) return e;
         k_attn_dq_tc<<<(unsigned)((int64_t)m.B * Hq * m.T), kBwdThreads, smem, s>>>(
-            tq, tk, tv, to, m, Hq, Hkv, scale, sl2, Drow, NL2, (__nv_bfloat16 *)dq, status);
+            tk, tv, (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)dO, m, Hq, Hkv, scale, sl2, Drow,
+            NL2, (__nv_bfloat16 *)dq, status);
     }
     return cudaGetLastError();
 }

@@ -99,6 +99,9 @@ __global__ void __launch_bounds__(kDmThreads, 3)
     const int64_t blk_stride = (int64_t)Hkv * bs * D;
     const int piece = lane & 15, par = lane >> 4;
     const int g = lane >> 2, t4 = lane & 3;
+    // chunks of one sub-piece: its ids (at most (chunks * 16 - 1) / bs + 2 of them)
+    // must fit the kDmMaxTps + 16 staged slots
+    const int32_t sub_chunks = bs >= kDmChunk ? kDmMaxTps : kDecMaxChunksPerCta * max(1, bs);
 
     int32_t b = rg.b0;
     int32_t pre = rg.pre_b0;
@@ -129,10 +132,11 @@ __global__ void __launch_bounds__(kDmThreads, 3)
         for (int i = 0; i < 16; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
         float mrow = -INFINITY, lrow = 0.f;  // row g (head g); rows g+8 are padding
 
-        // sub-pieces of at most kDecMaxChunksPerCta chunks: the table slice of each is
-        // staged in shared memory; the softmax state carries over
-        for (int32_t sp = ps; sp < pe; sp += kDecMaxChunksPerCta) {
-            const int32_t spe = min(pe, sp + kDecMaxChunksPerCta);
+        // sub-pieces whose table slice fits the kDmMaxTps + 16 ids staged in shared
+        // memory (72 chunks of 1-token blocks, 1152 of 16-token blocks); the softmax
+        // state carries over from one to the next
+        for (int32_t sp = ps; sp < pe; sp += sub_chunks) {
+            const int32_t spe = min(pe, sp + sub_chunks);
             const int32_t t_begin = (sp - cs) * kDecChunk;
             const int32_t t_end = min(ntok, (spe - cs) * kDecChunk);
             const int nchunks = (t_end - t_begin + kDmChunk - 1) / kDmChunk;
