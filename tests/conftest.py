@@ -36,14 +36,15 @@ def pytest_terminal_summary(terminalreporter):
         return
     fam = {}
     for what, flat, exc, tol in gu.REPORT:
-        key = what.split(" b")[0].split(" call")[0]
-        f0, e0, t0, n0 = fam.get(key, (0.0, -1e30, tol, 0))
-        fam[key] = (max(f0, flat), max(e0, exc), tol, n0 + 1)
+        # one row per check family and tolerance (bf16 and fp32 runs of a check apart)
+        key = (what.split(" b")[0].split(" call")[0], tol)
+        f0, e0, n0 = fam.get(key, (0.0, -1e30, 0))
+        fam[key] = (max(f0, flat), max(e0, exc), n0 + 1)
     tr = terminalreporter
     tr.write_sep("-", "parity: flat max-abs | excess beyond rounding | tolerance (checks)")
     for key in sorted(fam):
-        f, e, t, n = fam[key]
-        tr.write_line(f"{key[:48]:48s} {f:10.3g} {e:10.3g} {t:8.2g} ({n})")
+        f, e, n = fam[key]
+        tr.write_line(f"{key[0][:48]:48s} {f:10.3g} {e:10.3g} {key[1]:8.2g} ({n})")
     path = os.environ.get("KVS_PARITY_REPORT")
     if path:
         import json
