@@ -69,21 +69,16 @@ __global__ void k_bwd_prep(const __nv_bfloat16 *__restrict__ o, const __nv_bfloa
     }
 }
 
-// Store 64 fp32 values (times f) of a row as bf16 to 128 contiguous bytes.
-__device__ __forceinline__ void store_row64(__nv_bfloat16 *dst, const uint32_t (&a)[32],
-                                            const uint32_t (&b)[32], float f) {
+// Store 32 fp32 values (times f) of a row as bf16 to 64 contiguous bytes.
+__device__ __forceinline__ void store_row32(__nv_bfloat16 *dst, const uint32_t (&r)[32], float f) {
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        const uint32_t(&r)[32] = h ? b : a;
-#pragma unroll
-        for (int j = 0; j < 32; j += 8) {
-            uint4 w;
-            w.x = pack_bf16(__uint_as_float(r[j]) * f, __uint_as_float(r[j + 1]) * f);
-            w.y = pack_bf16(__uint_as_float(r[j + 2]) * f, __uint_as_float(r[j + 3]) * f);
-            w.z = pack_bf16(__uint_as_float(r[j + 4]) * f, __uint_as_float(r[j + 5]) * f);
-            w.w = pack_bf16(__uint_as_float(r[j + 6]) * f, __uint_as_float(r[j + 7]) * f);
-            *reinterpret_cast<uint4 *>(dst + h * 32 + j) = w;
-        }
+    for (int j = 0; j < 32; j += 8) {
+        uint4 w;
+        w.x = pack_bf16(__uint_as_float(r[j]) * f, __uint_as_float(r[j + 1]) * f);
+        w.y = pack_bf16(__uint_as_float(r[j + 2]) * f, __uint_as_float(r[j + 3]) * f);
+        w.z = pack_bf16(__uint_as_float(r[j + 4]) * f, __uint_as_float(r[j + 5]) * f);
+        w.w = pack_bf16(__uint_as_float(r[j + 6]) * f, __uint_as_float(r[j + 7]) * f);
+        *reinterpret_cast<uint4 *>(dst + j) = w;
     }
 }
 
@@ -92,11 +87,12 @@ __device__ __forceinline__ void store_row64(__nv_bfloat16 *dst, const uint32_t (
 //
 // An item is (128-row query tile of the key tile's column list, query head of
 // the group). TMEM: S^T [0,128) and dP^T [128,256) of the current item, dV
-// [256,384), dK [384,512). The eight elementwise warps split an item's rows in
-// two halves (warp group h takes rows 64h..64h+63, thread = key lane); each
-// writes its P^T (dS^T) as bf16 pairs into the first 32 of its own 64 columns
-// of S^T (dP^T), so neither half overwrites scores the other still reads. Per
-// item the tensor core runs, in issue order,
+// [256,384), dK [384,512). Sixteen elementwise warps (four per TMEM lane
+// quarter, so that each scheduler has four to hide the TMEM and exponential
+// latencies) split an item's rows in four parts (part p takes rows
+// 32p..32p+31, thread = key lane); each writes its P^T (dS^T) as bf16 pairs
+// into the first 16 of its own 32 columns of S^T (dP^T), so no part overwrites
+// scores another still reads. Per item the tensor core runs, in issue order,
 //   dV(n) += P^T(n) dO(n), S^T(n+1) = K Q(n+1)^T, dK(n) += dS^T(n) Q(n),
 //   dP^T(n+1) = V dO(n+1)^T
 // (four M=128 N=128 K=128 products): the elementwise phase P^T(n+1) runs while
@@ -105,7 +101,8 @@ __device__ __forceinline__ void store_row64(__nv_bfloat16 *dst, const uint32_t (
 // reads it (MMAs run in issue order) and after the elementwise warps reported
 // they had read it.
 
-constexpr int kBwdThreads = 320;  // warp 0 TMA, warp 1 MMA, warps 2..9 elementwise
+constexpr int kBwdEwThreads = 512;               // 16 elementwise warps
+constexpr int kBwdThreads = 64 + kBwdEwThreads;  // warp 0 TMA, warp 1 MMA, warps 2..17 elementwise
 // Q(n) is read by S^T(n) and dK(n), dO(n) by dP^T(n) and dV(n). With three Q
 // stages the load of Q(n+3) goes out when dK(n) completes, six products before
 // S^T(n+3); with two dO stages the load of dO(n+2) goes out when dV(n)
@@ -131,9 +128,9 @@ struct DkvSmem {
 // 1024-byte aligned (the swizzled tiles need it) instead of padding for it
 static_assert(sizeof(DkvSmem) <= 232448, "dK/dV shared memory over the 227 KB limit");
 
-// TMEM column of the bf16 pairs of rows 16kk..16kk+15 inside a 128-column region
-// whose halves hold rows 0..63 and 64..127 in their first 32 columns.
-__device__ __forceinline__ uint32_t packed_col(int kk) { return kk < 4 ? 8 * kk : 64 + 8 * (kk - 4); }
+// TMEM column of the bf16 pairs of rows (keys) 16kk..16kk+15 inside a 128-column
+// region whose four 32-column parts hold rows 32p..32p+31 in their first 16 columns.
+__device__ __forceinline__ uint32_t part_col(int kk) { return 32 * (kk >> 1) + 8 * (kk & 1); }
 
 __global__ void __launch_bounds__(kBwdThreads, 1)
     k_attn_dkdv_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -171,12 +168,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         for (int i = 0; i < kDkvRowStages; ++i) {
             mbar_init(&S.rfull[i], 1);
-            mbar_init(&S.rempty[i], 256);
+            mbar_init(&S.rempty[i], kBwdEwThreads);
         }
         mbar_init(&S.st_full, 1);
         mbar_init(&S.dp_full, 1);
-        mbar_init(&S.p_ready, 256);
-        mbar_init(&S.ds_ready, 256);
+        mbar_init(&S.p_ready, kBwdEwThreads);
+        mbar_init(&S.ds_ready, kBwdEwThreads);
         mbar_init(&S.acc_done, 1);
         mbar_init(&S.fin, 1);
         S.abort = 0;
@@ -285,7 +282,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
                     if (leader)
-                        mma_ts(tmem + cDV, tmem + cST + packed_col(kk), desc_add(om, kk * 2048), idMN,
+                        mma_ts(tmem + cDV, tmem + cST + part_col(kk), desc_add(om, kk * 2048), idMN,
                                kk > 0 ? 1u : acc);
                 if (leader) mma_commit(&S.oempty[n % kDkvOStages]);
                 const bool more = n + 1 < nw;
@@ -295,7 +292,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
                     if (leader)
-                        mma_ts(tmem + cDK, tmem + cDP + packed_col(kk), desc_add(qm, kk * 2048), idMN,
+                        mma_ts(tmem + cDK, tmem + cDP + part_col(kk), desc_add(qm, kk * 2048), idMN,
                                kk > 0 ? 1u : acc);
                 if (leader) mma_commit(&S.qempty[n % kDkvQStages]);
                 if (more && !issue_dp(n + 1)) break;
@@ -305,12 +302,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             wait_done(&S.fin, 0);
         }
     } else {
-        // thread = key row c (TMEM lane); group h takes query rows 64h..64h+63 of each item
-        const int quad = warp & 3, h = (warp - 2) >> 2;
+        // thread = key row c (TMEM lane); part p takes query rows 32p..32p+31 of each item
+        const int quad = warp & 3, part = (warp - 2) >> 2;
         const int c = quad * 32 + lane;
         const int j = k0 + c;
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-        const uint32_t colS = cST + h * 64, colP = cDP + h * 64;
+        const uint32_t colS = cST + part * 32, colP = cDP + part * 32;
         const int32_t kap = j < N ? m.kappa[(int64_t)b * N + j] : 0;
         bool ok = true;
         for (int n = 0; n < nw; ++n) {
@@ -320,16 +317,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 ok = false;
                 break;
             }
-            const int q0 = S.q0[s] + 64 * h;  // this group's first row
-            // visible query rows of this key among the group's 64: [rlo, rhi) (j <= t < kappa_j)
-            int rlo = 0, rhi = 64;
+            const int q0 = S.q0[s] + 32 * part;  // this part's first row
+            // visible query rows of this key among the part's 32: [rlo, rhi) (j <= t < kappa_j)
+            int rlo = 0, rhi = 32;
             if (!S.full_tile[s]) {
                 if (j >= N) {
                     rlo = rhi = 0;
                 } else {
                     const int64_t lo = (int64_t)j - q0, hi = (int64_t)(kap < N ? kap : N) - q0;
-                    rlo = (int)(lo < 0 ? 0 : (lo > 64 ? 64 : lo));
-                    rhi = (int)(hi < 0 ? 0 : (hi > 64 ? 64 : hi));
+                    rlo = (int)(lo < 0 ? 0 : (lo > 32 ? 32 : lo));
+                    rhi = (int)(hi < 0 ? 0 : (hi > 32 ? 32 : hi));
                 }
             }
             if (!warp_wait(&S.st_full, ph, abort, status)) {
@@ -337,50 +334,34 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 break;
             }
             tc_fence_after();
-            // P^T = 2^(S^T c - LSE_t log2 e), kept only as bf16 pairs (the values the
-            // dV MMA consumes)
-            uint32_t pk[32];
+            // P^T = 2^(S^T c - LSE_t log2 e), kept in fp32 for dS^T and stored as
+            // bf16 pairs (the A operand of dV)
+            float pf[32];
             {
-                uint32_t r0[32], r1[32];
+                uint32_t r0[32], pk[16];
                 tmem_ld32(tmem + lane_off + colS, r0);
-                tmem_ld32(tmem + lane_off + colS + 32, r1);
                 tmem_ld_wait();
-                const float4 *l2v = reinterpret_cast<const float4 *>(S.nl2[s] + 64 * h);
-                const bool all_vis = rlo <= 0 && rhi >= 64;
-                if (__all_sync(0xffffffffu, all_vis)) {
+                const float4 *l2v = reinterpret_cast<const float4 *>(S.nl2[s] + 32 * part);
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const float4 lv = l2v[i];
-                        const int rr = 4 * i;
-                        const float a0 = __uint_as_float(rr < 32 ? r0[rr] : r1[rr - 32]);
-                        const float a1 = __uint_as_float(rr < 32 ? r0[rr + 1] : r1[rr - 31]);
-                        const float a2 = __uint_as_float(rr < 32 ? r0[rr + 2] : r1[rr - 30]);
-                        const float a3 = __uint_as_float(rr < 32 ? r0[rr + 3] : r1[rr - 29]);
-                        // half of the exponentials on the FMA pipe, half on the SFU
-                        float x0, x1, x2, x3, e0, e1;
-                        fma2v(a0, a1, scale_log2, lv.x, lv.y, x0, x1);
-                        fma2v(a2, a3, scale_log2, lv.z, lv.w, x2, x3);
-                        exp2_fma_x2(x0, x1, e0, e1);
-                        pk[2 * i] = pack_bf16(e0, e1);
-                        pk[2 * i + 1] = pack_bf16(ex2(x2), ex2(x3));
-                    }
-                } else {
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const float4 lv = l2v[i];
-                        const float ls[4] = {lv.x, lv.y, lv.z, lv.w};
-                        float q4[4];
-#pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            const int rr = 4 * i + u;
-                            const float a = __uint_as_float(rr < 32 ? r0[rr] : r1[rr - 32]);
-                            q4[u] = (rr >= rlo && rr < rhi) ? ex2(fmaf(a, scale_log2, ls[u])) : 0.f;
-                        }
-                        pk[2 * i] = pack_bf16(q4[0], q4[1]);
-                        pk[2 * i + 1] = pack_bf16(q4[2], q4[3]);
-                    }
+                for (int i = 0; i < 8; ++i) {
+                    const float4 lv = l2v[i];
+                    // half of the exponentials on the FMA pipe, half on the SFU
+                    float x0, x1, x2, x3;
+                    fma2v(__uint_as_float(r0[4 * i]), __uint_as_float(r0[4 * i + 1]), scale_log2, lv.x, lv.y,
+                          x0, x1);
+                    fma2v(__uint_as_float(r0[4 * i + 2]), __uint_as_float(r0[4 * i + 3]), scale_log2, lv.z,
+                          lv.w, x2, x3);
+                    exp2_fma_x2(x0, x1, pf[4 * i], pf[4 * i + 1]);
+                    pf[4 * i + 2] = ex2(x2);
+                    pf[4 * i + 3] = ex2(x3);
                 }
-                tmem_st32(tmem + lane_off + colS, pk);
+                if (__any_sync(0xffffffffu, rlo > 0 || rhi < 32)) {
+#pragma unroll
+                    for (int rr = 0; rr < 32; ++rr) pf[rr] = (rr >= rlo && rr < rhi) ? pf[rr] : 0.f;
+                }
+#pragma unroll
+                for (int i = 0; i < 16; ++i) pk[i] = pack_bf16(pf[2 * i], pf[2 * i + 1]);
+                tmem_st16(tmem + lane_off + colS, pk);
             }
             tmem_st_wait();
             tc_fence_before();
@@ -390,54 +371,49 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 break;
             }
             tc_fence_after();
-            // dS^T = P^T (dP^T - D_t), from the bf16 P^T above
+            // dS^T = P^T (dP^T - D_t)
             {
-                uint32_t r0[32], r1[32], dk2[32];
+                uint32_t r0[32], dk2[16];
                 tmem_ld32(tmem + lane_off + colP, r0);
-                tmem_ld32(tmem + lane_off + colP + 32, r1);
                 tmem_ld_wait();
-                const float4 *ddv = reinterpret_cast<const float4 *>(S.dd[s] + 64 * h);
+                const float4 *ddv = reinterpret_cast<const float4 *>(S.dd[s] + 32 * part);
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
+                for (int i = 0; i < 8; ++i) {
                     const float4 dv4 = ddv[i];
-                    const int rr = 4 * i;
-                    const float a0 = __uint_as_float(rr < 32 ? r0[rr] : r1[rr - 32]);
-                    const float a1 = __uint_as_float(rr < 32 ? r0[rr + 1] : r1[rr - 31]);
-                    const float a2 = __uint_as_float(rr < 32 ? r0[rr + 2] : r1[rr - 30]);
-                    const float a3 = __uint_as_float(rr < 32 ? r0[rr + 3] : r1[rr - 29]);
                     float d0, d1, d2, d3;
-                    f2_split(f2_mul(f2_make(bf16_lo(pk[2 * i]), bf16_hi(pk[2 * i])),
-                                    f2_sub(f2_make(a0, a1), f2_make(dv4.x, dv4.y))), d0, d1);
-                    f2_split(f2_mul(f2_make(bf16_lo(pk[2 * i + 1]), bf16_hi(pk[2 * i + 1])),
-                                    f2_sub(f2_make(a2, a3), f2_make(dv4.z, dv4.w))), d2, d3);
+                    f2_split(f2_mul(f2_make(pf[4 * i], pf[4 * i + 1]),
+                                    f2_sub(f2_make(__uint_as_float(r0[4 * i]), __uint_as_float(r0[4 * i + 1])),
+                                           f2_make(dv4.x, dv4.y))), d0, d1);
+                    f2_split(f2_mul(f2_make(pf[4 * i + 2], pf[4 * i + 3]),
+                                    f2_sub(f2_make(__uint_as_float(r0[4 * i + 2]), __uint_as_float(r0[4 * i + 3])),
+                                           f2_make(dv4.z, dv4.w))), d2, d3);
                     dk2[2 * i] = pack_bf16(d0, d1);
                     dk2[2 * i + 1] = pack_bf16(d2, d3);
                 }
-                tmem_st32(tmem + lane_off + colP, dk2);
+                tmem_st16(tmem + lane_off + colP, dk2);
             }
             tmem_st_wait();
             tc_fence_before();
             mbar_arrive(&S.ds_ready);
             mbar_arrive(&S.rempty[s]);  // done with this item's row data
         }
-        // each group writes 64 of the 128 dimensions of dV and dK
-        const uint32_t col0 = h * 64;
+        // each part writes 32 of the 128 dimensions of dV and dK
+        const uint32_t col0 = part * 32;
         if (ok && nw > 0 && warp_wait(&S.acc_done, 0, abort, status)) {
             tc_fence_after();
             const int64_t ro = (((int64_t)b * N + j) * Hkv + kvh) * 128 + col0;
 #pragma unroll
             for (int which = 0; which < 2; ++which) {
-                uint32_t r0[32], r1[32];
-                const uint32_t cb = (which ? cDK : cDV) + col0;
-                tmem_ld32(tmem + lane_off + cb, r0);
-                tmem_ld32(tmem + lane_off + cb + 32, r1);
+                uint32_t r0[32];
+                const float f = which ? scale : 1.f;
+                tmem_ld32(tmem + lane_off + (which ? cDK : cDV) + col0, r0);
                 tmem_ld_wait();
-                if (j < N) store_row64((which ? dk : dv) + ro, r0, r1, which ? scale : 1.f);
+                if (j < N) store_row32((which ? dk : dv) + ro, r0, f);
             }
         } else if (nw == 0 && j < N) {
             // a key no query sees (cannot happen for a valid mask: the diagonal is visible)
             const int64_t ro = (((int64_t)b * N + j) * Hkv + kvh) * 128 + col0;
-            for (int i = 0; i < 64; i += 8) {
+            for (int i = 0; i < 32; i += 8) {
                 *reinterpret_cast<uint4 *>(dk + ro + i) = make_uint4(0, 0, 0, 0);
                 *reinterpret_cast<uint4 *>(dv + ro + i) = make_uint4(0, 0, 0, 0);
             }
@@ -455,10 +431,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 // [384,448) and dO [448,512) as bf16 pairs: S = Q K^T and dP = dO V^T take
 // their A operand from TMEM, so each product reads only K or V from shared
 // memory (160 KB of shared-memory reads and fills per item instead of 224 KB,
-// below the 1536 cycles of tensor work). The eight elementwise warps split an
-// item's 128 keys in two halves (thread = query row); each writes its dS as
-// bf16 pairs into the first 32 of its own 64 columns of dP, the A operand of
-// dQ += dS K. Per item the tensor core runs, in issue order, dP(n),
+// below the 1536 cycles of tensor work). Sixteen elementwise warps (four per
+// TMEM lane quarter, so that each scheduler has four to hide the TMEM and
+// exponential latencies) split an item's 128 keys in four parts of 32 (thread =
+// query row); each writes its dS as bf16 pairs into the first 16 of its own 32
+// columns of dP, the A operand of dQ += dS K. Per item the tensor core runs, in issue order, dP(n),
 // [S(n) read] S(n+1), [dS(n) written] dQ(n), then dP(n+1): each product that
 // overwrites a TMEM region comes after the one that reads it.
 //
@@ -507,11 +484,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             mbar_init(&S.vfull[i], 1);
             mbar_init(&S.vempty[i], 1);
         }
-        mbar_init(&S.qo_ready, 256);
+        mbar_init(&S.qo_ready, kBwdEwThreads);
         mbar_init(&S.s_full, 1);
         mbar_init(&S.dp_full, 1);
-        mbar_init(&S.s_free, 256);
-        mbar_init(&S.ds_ready, 256);
+        mbar_init(&S.s_free, kBwdEwThreads);
+        mbar_init(&S.ds_ready, kBwdEwThreads);
         mbar_init(&S.acc_done, 1);
         mbar_init(&S.fin, 1);
         S.abort = 0;
@@ -608,7 +585,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
                     if (leader)
-                        mma_ts(tmem + cDQ, tmem + cDP + packed_col(kk), desc_add(km, kk * 2048), idMN,
+                        mma_ts(tmem + cDQ, tmem + cDP + part_col(kk), desc_add(km, kk * 2048), idMN,
                                kk > 0 ? 1u : acc);
                 if (leader) mma_commit(&S.kempty[n % kDqKStages]);
                 // dP(n+1) overwrites dS(n) after dQ(n) has read it (in issue order)
@@ -619,32 +596,33 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             wait_done(&S.fin, 0);
         }
     } else {
-        // thread = query row (TMEM lane); half = which 64 key columns it handles
-        const int quad = warp & 3, half = (warp - 2) >> 2;
+        // thread = query row (TMEM lane); part = which 32 key columns (and which 32
+        // dimensions of Q, dO and dQ) it handles
+        const int quad = warp & 3, part = (warp - 2) >> 2;
         const int row = quad * 32 + lane;
         const int t = q0 + row;
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-        const uint32_t col0 = half * 64;
+        const uint32_t col0 = part * 32;
         const int64_t ro = ((int64_t)b * Hq + hq) * Tpad + t;
         const float nl2 = NL2[ro], dd = Drow[ro];
         const uint64_t dd2 = f2_make(dd, dd);
         bool ok = true;
         if (nt > 0) {
-            // this row's half of Q and of dO into TMEM as bf16 pairs (the A operands);
+            // this row's part of Q and of dO into TMEM as bf16 pairs (the A operands);
             // rows past N are zero
-            uint32_t r[32];
+            uint32_t r[16];
 #pragma unroll
             for (int w = 0; w < 2; ++w) {
-                const __nv_bfloat16 *src = (w ? dO : q) + (((int64_t)b * N + t) * Hq + hq) * 128 + half * 64;
+                const __nv_bfloat16 *src = (w ? dO : q) + (((int64_t)b * N + t) * Hq + hq) * 128 + col0;
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
+                for (int i = 0; i < 4; ++i) {
                     const uint4 u = t < N ? *reinterpret_cast<const uint4 *>(src + 8 * i) : make_uint4(0, 0, 0, 0);
                     r[4 * i] = u.x;
                     r[4 * i + 1] = u.y;
                     r[4 * i + 2] = u.z;
                     r[4 * i + 3] = u.w;
                 }
-                tmem_st32(tmem + lane_off + (w ? cO : cQ) + half * 32, r);
+                tmem_st16(tmem + lane_off + (w ? cO : cQ) + part * 16, r);
             }
             tmem_st_wait();
             tc_fence_before();
@@ -659,47 +637,34 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 break;
             }
             const bool partial = S.pid[ks] >= 0;  // same for the whole CTA
-            uint2 bits = make_uint2(~0u, ~0u);
-            if (partial) bits = *reinterpret_cast<const uint2 *>(&S.bits[ks][row * 4 + half * 2]);
+            const uint32_t bits = partial ? S.bits[ks][row * 4 + part] : ~0u;
             if (!warp_wait(&S.s_full, n & 1, abort, status)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            // P = 2^(S c - LSE log2 e) for this thread's 64 key columns, kept as bf16
-            // pairs; dS = P (dP - D) then rounds to bf16 for the dQ MMA
-            uint32_t pp[32];
+            // P = 2^(S c - LSE log2 e) for this thread's 32 key columns, kept in fp32;
+            // dS = P (dP - D) then rounds to bf16 for the dQ MMA
+            float pf[32];
             {
-                uint32_t r0[32], r1[32];
+                uint32_t r0[32];
                 tmem_ld32(tmem + lane_off + cS + col0, r0);
-                tmem_ld32(tmem + lane_off + cS + col0 + 32, r1);
                 tmem_ld_wait();
                 tc_fence_before();
                 mbar_arrive(&S.s_free);
-                if (!partial) {
 #pragma unroll
-                    for (int jj = 0; jj < 32; jj += 2) {
-                        // first 32 columns on the FMA pipe, last 32 on the SFU
-                        float x0, x1, x2, x3, e0, e1;
-                        fma2(__uint_as_float(r0[jj]), __uint_as_float(r0[jj + 1]), scale_log2, nl2, x0, x1);
-                        fma2(__uint_as_float(r1[jj]), __uint_as_float(r1[jj + 1]), scale_log2, nl2, x2, x3);
-                        exp2_fma_x2(x0, x1, e0, e1);
-                        pp[jj >> 1] = pack_bf16(e0, e1);
-                        pp[16 + (jj >> 1)] = pack_bf16(ex2(x2), ex2(x3));
-                    }
-                } else {
+                for (int jj = 0; jj < 32; jj += 4) {
+                    // two columns of each four on the FMA pipe, two on the SFU
+                    float x0, x1, x2, x3;
+                    fma2(__uint_as_float(r0[jj]), __uint_as_float(r0[jj + 1]), scale_log2, nl2, x0, x1);
+                    fma2(__uint_as_float(r0[jj + 2]), __uint_as_float(r0[jj + 3]), scale_log2, nl2, x2, x3);
+                    exp2_fma_x2(x0, x1, pf[jj], pf[jj + 1]);
+                    pf[jj + 2] = ex2(x2);
+                    pf[jj + 3] = ex2(x3);
+                }
+                if (partial) {
 #pragma unroll
-                    for (int jj = 0; jj < 32; jj += 2) {
-                        float x0, x1, x2, x3, e0, e1;
-                        fma2(__uint_as_float(r0[jj]), __uint_as_float(r0[jj + 1]), scale_log2, nl2, x0, x1);
-                        fma2(__uint_as_float(r1[jj]), __uint_as_float(r1[jj + 1]), scale_log2, nl2, x2, x3);
-                        exp2_fma_x2(x0, x1, e0, e1);
-                        const float e2 = ex2(x2), e3 = ex2(x3);
-                        pp[jj >> 1] = pack_bf16(((bits.x >> jj) & 1u) ? e0 : 0.f,
-                                                ((bits.x >> (jj + 1)) & 1u) ? e1 : 0.f);
-                        pp[16 + (jj >> 1)] = pack_bf16(((bits.y >> jj) & 1u) ? e2 : 0.f,
-                                                       ((bits.y >> (jj + 1)) & 1u) ? e3 : 0.f);
-                    }
+                    for (int jj = 0; jj < 32; ++jj) pf[jj] = ((bits >> jj) & 1u) ? pf[jj] : 0.f;
                 }
             }
             if (!warp_wait(&S.dp_full, n & 1, abort, status)) {
@@ -708,25 +673,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             }
             tc_fence_after();
             {
-                uint32_t r0[32], r1[32], pk[32];
+                uint32_t r0[32], pk[16];
                 tmem_ld32(tmem + lane_off + cDP + col0, r0);
-                tmem_ld32(tmem + lane_off + cDP + col0 + 32, r1);
                 tmem_ld_wait();
 #pragma unroll
                 for (int jj = 0; jj < 32; jj += 2) {
-                    float d0, d1, d2, d3;
-                    const uint32_t pa = pp[jj >> 1], pb = pp[16 + (jj >> 1)];
-                    f2_split(f2_mul(f2_make(bf16_lo(pa), bf16_hi(pa)),
+                    float d0, d1;
+                    f2_split(f2_mul(f2_make(pf[jj], pf[jj + 1]),
                                     f2_sub(f2_make(__uint_as_float(r0[jj]), __uint_as_float(r0[jj + 1])), dd2)),
                              d0, d1);
-                    f2_split(f2_mul(f2_make(bf16_lo(pb), bf16_hi(pb)),
-                                    f2_sub(f2_make(__uint_as_float(r1[jj]), __uint_as_float(r1[jj + 1])), dd2)),
-                             d2, d3);
                     pk[jj >> 1] = pack_bf16(d0, d1);
-                    pk[16 + (jj >> 1)] = pack_bf16(d2, d3);
                 }
-                // keys col0..col0+63 as bf16 pairs in the first 32 columns of this half
-                tmem_st32(tmem + lane_off + cDP + col0, pk);
+                // keys col0..col0+31 as bf16 pairs in the first 16 columns of this part
+                tmem_st16(tmem + lane_off + cDP + col0, pk);
             }
             tmem_st_wait();
             tc_fence_before();
@@ -734,11 +693,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         if (ok && nt > 0 && warp_wait(&S.acc_done, 0, abort, status)) {
             tc_fence_after();
-            uint32_t r0[32], r1[32];
+            uint32_t r0[32];
             tmem_ld32(tmem + lane_off + cDQ + col0, r0);
-            tmem_ld32(tmem + lane_off + cDQ + col0 + 32, r1);
             tmem_ld_wait();
-            if (t < N) store_row64(dq + (((int64_t)b * N + t) * Hq + hq) * 128 + col0, r0, r1, scale);
+            if (t < N) store_row32(dq + (((int64_t)b * N + t) * Hq + hq) * 128 + col0, r0, scale);
         }
     }
     tc_fence_before();
