@@ -345,13 +345,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
                     const float4 lv = l2v[i];
-                    // half of the exponentials on the FMA pipe, half on the SFU
+                    // a quarter of the exponentials on the FMA pipe, the rest on the SFU
                     float x0, x1, x2, x3;
                     fma2v(__uint_as_float(r0[4 * i]), __uint_as_float(r0[4 * i + 1]), scale_log2, lv.x, lv.y,
                           x0, x1);
                     fma2v(__uint_as_float(r0[4 * i + 2]), __uint_as_float(r0[4 * i + 3]), scale_log2, lv.z,
                           lv.w, x2, x3);
-                    exp2_fma_x2(x0, x1, pf[4 * i], pf[4 * i + 1]);
+                    if (i & 1) {
+                        exp2_fma_x2(x0, x1, pf[4 * i], pf[4 * i + 1]);
+                    } else {
+                        pf[4 * i] = ex2(x0);
+                        pf[4 * i + 1] = ex2(x1);
+                    }
                     pf[4 * i + 2] = ex2(x2);
                     pf[4 * i + 3] = ex2(x3);
                 }
@@ -654,11 +659,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 mbar_arrive(&S.s_free);
 #pragma unroll
                 for (int jj = 0; jj < 32; jj += 4) {
-                    // two columns of each four on the FMA pipe, two on the SFU
+                    // a quarter of the exponentials on the FMA pipe, the rest on the SFU
                     float x0, x1, x2, x3;
                     fma2(__uint_as_float(r0[jj]), __uint_as_float(r0[jj + 1]), scale_log2, nl2, x0, x1);
                     fma2(__uint_as_float(r0[jj + 2]), __uint_as_float(r0[jj + 3]), scale_log2, nl2, x2, x3);
-                    exp2_fma_x2(x0, x1, pf[jj], pf[jj + 1]);
+                    if ((jj >> 2) & 1) {
+                        exp2_fma_x2(x0, x1, pf[jj], pf[jj + 1]);
+                    } else {
+                        pf[jj] = ex2(x0);
+                        pf[jj + 1] = ex2(x1);
+                    }
                     pf[jj + 2] = ex2(x2);
                     pf[jj + 3] = ex2(x3);
                 }
