@@ -374,7 +374,7 @@ def _durations(rec):
 # 1/16-scale bs1 workload: kernel -> (bytes of that launch, visible pairs x query heads it processed,
 # sha1 prefix of the kernel sources it was taken with). The bench scales it to its own launch by the
 # pairs processed and reports null once the sources have changed.
-TRAFFIC = {"dkdv": (1.671485e9 + 57.177344e6, 27713931 * 64, "21c8d7eef322")}
+TRAFFIC = {"dkdv": (1.791634e9 + 59.25888e6, 27713931 * 64, "5d4bf2f36424")}
 
 
 def _src_hash(files):
