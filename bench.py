@@ -297,8 +297,10 @@ class Step:
         mask = 2 * (3 + has_ev) + 2        # count call + fill call (+ 2 fill kernels)
         return mask + 2 + 1 + 3 + 2 + 1 + 1 + 1 + 1
 
-    def run(self, ev_rec=None):
-        """One step; if ev_rec is a dict, records CUDA events around each call."""
+    def run(self, ev_rec=None, bwd_wait=None):
+        """One step; if ev_rec is a dict, records CUDA events around each call. With
+        bwd_wait (a CUDA event) the backward waits for it: the forward may start
+        while dO is still being copied in."""
         kvs, cfg = self.kvs, self.cfg
         B, N, Hq, Hkv, d = cfg.batch, cfg.n_tokens, cfg.hq, cfg.hkv, cfg.d
 
@@ -317,6 +319,8 @@ class Step:
         kvs.kvs_masked_attn_fwd(self.q, self.k, self.v, mask, cfg.scale, out=self.o, lse=self.lse,
                                 out_lo=self.o_lo, status=self.status)
         mark("fwd")
+        if bwd_wait is not None:
+            torch.cuda.current_stream().wait_event(bwd_wait)
         for st, name in ((kvs.KVS_BWD_PREP, "bwd_prep"), (kvs.KVS_BWD_DKDV, "dkdv"), (kvs.KVS_BWD_DQ, "dq")):
             kvs.kvs_masked_attn_bwd(self.q, self.k, self.v, self.o, self.do, self.lse, mask, cfg.scale,
                                     dq=self.dq, dk=self.dk, dv=self.dv, ws=self.bwd_ws, status=self.status,
@@ -801,7 +805,8 @@ def run_ours(args):
         print(json.dumps(line), flush=True)
 
 
-IN_NAMES = ("q_raw", "k_raw", "v", "do", "events")     # a step's inputs
+IN_NAMES = ("events", "q_raw", "k_raw", "v", "do")     # a step's inputs (copied in this order)
+N_FWD_IN = 4                                             # the first four feed the forward
 OUT_NAMES = ("dq_raw", "dk_raw", "dv", "o_dec")          # a step's results
 
 
@@ -809,10 +814,11 @@ def _e2e(step, args, flops_step):
     """Every step copies its inputs (raw q, k, v, dO, event log) from pinned host
     memory and reads its results (dq, dk in the pre-RoPE basis, dv, the decode
     output) back, timed with CUDA events from the first copy in to the last copy
-    out. Steps are pipelined as a serving or training loop would run them: two
-    sets of device inputs and results, the copy of step i+1's inputs on one copy
-    stream and of step i-1's results on another while step i computes; a set is
-    refilled only after the step that read it has finished."""
+    out. Steps are pipelined as a training loop would run them: two sets of device
+    inputs and results, the copy of step i+1's inputs on one copy stream and of
+    step i-1's results on another while step i computes; a set is refilled only
+    after the step that read it has finished. Within a step the forward starts once
+    its inputs (event log, q, k, v) are in; the backward also waits for dO."""
     ins = [getattr(step, n) for n in IN_NAMES]
     outs = [getattr(step, n) for n in OUT_NAMES]
     h_in = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in ins]
@@ -825,6 +831,7 @@ def _e2e(step, args, flops_step):
     h2d, d2h = torch.cuda.Stream(), torch.cuda.Stream()
     ev = lambda: torch.cuda.Event()
     in_ready, in_free, out_ready, out_free = [ev(), ev()], [ev(), ev()], [ev(), ev()], [ev(), ev()]
+    fwd_ready = [ev(), ev()]
     s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
     s.record(h2d)
@@ -834,15 +841,17 @@ def _e2e(step, args, flops_step):
         with torch.cuda.stream(h2d):
             if i >= 2:
                 h2d.wait_event(in_free[k])
-            for h, t in zip(h_in, s_in):
+            for j, (h, t) in enumerate(zip(h_in, s_in)):
                 t.copy_(h, non_blocking=True)
+                if j == N_FWD_IN - 1:
+                    fwd_ready[k].record(h2d)
             in_ready[k].record(h2d)
-        comp.wait_event(in_ready[k])
+        comp.wait_event(fwd_ready[k])
         if i >= 2:
             comp.wait_event(out_free[k])
         for nm, t in zip(IN_NAMES + OUT_NAMES, s_in + s_out):
             setattr(step, nm, t)
-        step.run()
+        step.run(bwd_wait=in_ready[k])
         in_free[k].record(comp)
         out_ready[k].record(comp)
         with torch.cuda.stream(d2h):
@@ -863,7 +872,8 @@ def _e2e(step, args, flops_step):
     return {"value": flops_step / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
             "h2d_bytes_per_step": int(sum(t.numel() * t.element_size() for t in ins)),
             "d2h_bytes_per_step": int(sum(t.numel() * t.element_size() for t in outs)),
-            "ms_per_step": ms, "steps": n, "pipelined": "copies of step i+1 in and i-1 out overlap step i"}
+            "ms_per_step": ms, "steps": n,
+            "pipelined": "copies of step i+1 in and i-1 out overlap step i; dO's copy overlaps the forward"}
 
 
 def main():
