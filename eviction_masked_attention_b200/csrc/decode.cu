@@ -273,12 +273,34 @@ cudaError_t launch_decode_mma(int G, const void *q, const void *kc, const void *
 // Merge the partials of one (sequence, query head): thread e owns output dim e.
 // The unit's pieces sit in the CTAs of its first and last chunk and the ones
 // between; a unit held by one CTA was written by it directly, one without live
-// entries gets zeros.
+// entries gets zeros. The pieces' maxima and sums are read by the block in
+// parallel (one piece per thread) and reduced; each piece's weight 2^(m - M)
+// goes to shared memory, and every thread then sums its dimension over the
+// pieces with independent loads.
+template <int D>
+__device__ __forceinline__ float block_reduce(float v, bool is_max, float *s_red) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const float w = __shfl_xor_sync(0xffffffffu, v, o);
+        v = is_max ? fmaxf(v, w) : v + w;
+    }
+    __syncthreads();  // s_red is free (a previous reduction has been read)
+    if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = v;
+    __syncthreads();
+    float r = s_red[0];
+#pragma unroll
+    for (int w = 1; w < D / 32; ++w) r = is_max ? fmaxf(r, s_red[w]) : r + s_red[w];
+    return r;
+}
+
 template <typename T, int D>
 __global__ void __launch_bounds__(D)
     k_decode_combine(const int32_t *__restrict__ num_tokens, int32_t B, int32_t Hq, int32_t Hkv,
                      int32_t cap, int64_t n_cta, const int64_t *__restrict__ pre_ws,
                      const float *__restrict__ partials, T *__restrict__ o) {
+    static_assert(D % 32 == 0 && D >= 32, "whole warps");
+    __shared__ float s_w[kDecWave];  // weight of each piece (at most one per CTA)
+    __shared__ float s_red[D / 32];
     const int h = blockIdx.x, b = blockIdx.y, e = threadIdx.x;
     const int G = Hq / Hkv, kvh = h / G, g = h % G;
     const int64_t nch = dec_nch(dec_ntok(num_tokens, b, cap));
@@ -294,21 +316,29 @@ __global__ void __launch_bounds__(D)
     const int64_t u = (int64_t)b * Hkv + kvh;
     // With at least as many chunks as CTAs every CTA in [c_first, c_last] holds a
     // piece of the unit. With fewer, each CTA holds at most one chunk, and the
-    // unit's pieces are the CTAs of its chunks.
+    // unit's pieces are the CTAs of its chunks. Either way there are at most
+    // n_cta <= kDecWave pieces.
     const bool per_chunk = tc < n_cta;
-    const int64_t n_it = per_chunk ? nch : c_last - c_first + 1;
-    auto slot = [&](int64_t i) { return (per_chunk ? dec_cta_of(cs + i, tc, n_cta) : c_first + i) + u; };
-    float M = -INFINITY;
-    for (int64_t i = 0; i < n_it; ++i) M = fmaxf(M, partials[(slot(i) * G + g) * (D + 2) + D]);
+    const int n_it = (int)(per_chunk ? nch : c_last - c_first + 1);
+    auto row = [&](int i) {
+        const int64_t slot = (per_chunk ? dec_cta_of(cs + i, tc, n_cta) : c_first + i) + u;
+        return partials + (slot * G + g) * (D + 2);
+    };
+    float mloc = -INFINITY;
+    for (int i = e; i < n_it; i += D) mloc = fmaxf(mloc, row(i)[D]);
+    const float M = block_reduce<D>(mloc, true, s_red);
     const float Mr = M == -INFINITY ? 0.f : M;
-    float L = 0.f, A = 0.f;
-#pragma unroll 4
-    for (int64_t i = 0; i < n_it; ++i) {
-        const float *pp = partials + (slot(i) * G + g) * (D + 2);
+    float lloc = 0.f;
+    for (int i = e; i < n_it; i += D) {
+        const float *pp = row(i);
         const float f = ex2(pp[D] - Mr);
-        L += pp[D + 1] * f;
-        A += pp[e] * f;
+        s_w[i] = f;
+        lloc += pp[D + 1] * f;
     }
+    const float L = block_reduce<D>(lloc, false, s_red);  // its barriers also publish s_w
+    float A = 0.f;
+#pragma unroll 8
+    for (int i = 0; i < n_it; ++i) A += row(i)[e] * s_w[i];
     store_out(o, oi, L > 0.f ? A / L : 0.f);
 }
 
