@@ -396,7 +396,7 @@ extern "C" kvs_status kvs_paged_decode_attn(const void *q, const void *k_cache, 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     cudaError_t e = cudaSuccess;
     if (bf) {
-        // bf16: bulk-copy staging + warp-level tensor-core products
+        // bf16: cp.async staging + warp-level tensor-core products
         e = launch_decode_mma(G, q, k_cache, v_cache, block_table, num_tokens, B, Hq, Hkv,
                               block_size, max_blocks, pool_blocks, qs, p.ctas, pre, part, o,
                               dev_status, s);
