@@ -611,7 +611,10 @@ __global__ void __launch_bounds__(kFwd2Threads, 1)
 //
 // The same schedule as k_attn_fwd_tc2 with the softmax reading each S tile in
 // one pass: all 128 score columns of a row come into registers with a single
-// TMEM round trip (about 194 registers per softmax thread). The block has three
+// TMEM round trip (about 194 registers per softmax thread). P is handed to the
+// MMA warp in two halves of 64 keys: PV's first four k-steps run while the
+// softmax still computes the second half, which shortens each head's
+// S -> softmax -> PV -> next S chain. The block has three
 // warpgroups of 128 threads -- warp 0 TMA, warp 1 MMA, warps 2-3 idle; warps
 // 4-7 head h0; warps 8-11 head h0+1 -- launched at 168 registers per thread;
 // after set-up the first warpgroup gives registers back (setmaxnreg.dec to 88)
@@ -632,7 +635,8 @@ struct Fwd3Smem {  // as Fwd2Smem, plus the skip flag
     // softmax groups finished tile n+1 and so tile n
     uint32_t bits[4][128 * 4];
     int32_t pid[4];             // partial index of the tile in each bit stage (-1: full)
-    uint64_t bar_q, kfull[2], kempty[2], vfull[2], vempty[2], sfull[2], pfull[2], odone[2], bfull[4], fin;
+    // pfull[x][hc]: head x's P for keys 64hc..64hc+63 is in TMEM
+    uint64_t bar_q, kfull[2], kempty[2], vfull[2], vempty[2], sfull[2], pfull[2][2], odone[2], bfull[4], fin;
     uint32_t tmem_base;
     int abort;
     int skip;
@@ -666,7 +670,8 @@ __global__ void __launch_bounds__(kFwd3Threads, 1)
             mbar_init(&S.vfull[i], 1);
             mbar_init(&S.vempty[i], 1);
             mbar_init(&S.sfull[i], 1);
-            mbar_init(&S.pfull[i], 128);
+            mbar_init(&S.pfull[i][0], 128);
+            mbar_init(&S.pfull[i][1], 128);
             mbar_init(&S.odone[i], 1);
         }
         for (int i = 0; i < 4; ++i) mbar_init(&S.bfull[i], 1);
@@ -743,13 +748,21 @@ __global__ void __launch_bounds__(kFwd3Threads, 1)
                 }
                 if (leader) mma_commit(&S.sfull[x]);
             };
-            auto issue_pv = [&](int x, int n) {
+            // PV(n) of head x in two halves of 64 keys, each issued once the softmax
+            // has written that half of P
+            auto issue_pv = [&](int x, int n) -> bool {
                 const uint64_t vd = (n & 1) ? vd1 : vd0;
                 const uint32_t d = tmem + 256 + x * 128, pa = tmem + x * 128, acc = n > 0 ? 1u : 0u;
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    if (leader) mma_ts(d, pa + kk * 8, desc_add(vd, kk * 2048), idPV, kk > 0 ? 1u : acc);
+                for (int hc = 0; hc < 2; ++hc) {
+                    if (!warp_wait(&S.pfull[x][hc], n & 1, abort, status)) return false;
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 4 * hc; kk < 4 * hc + 4; ++kk)
+                        if (leader) mma_ts(d, pa + kk * 8, desc_add(vd, kk * 2048), idPV, kk > 0 ? 1u : acc);
+                }
                 if (leader) mma_commit(&S.odone[x]);
+                return true;
             };
             bool ok = warp_wait(&S.bar_q, 0, abort, status) &&
                       warp_wait(&S.kfull[0], 0, abort, status);
@@ -762,18 +775,14 @@ __global__ void __launch_bounds__(kFwd3Threads, 1)
             for (int n = 0; ok && n < nt; ++n) {
                 const int s = n & 1;
                 const bool more = n + 1 < nt;
-                if (!warp_wait(&S.pfull[0], n & 1, abort, status)) break;
                 if (!warp_wait(&S.vfull[s], (n >> 1) & 1, abort, status)) break;
-                tc_fence_after();
-                issue_pv(0, n);
+                if (!issue_pv(0, n)) break;
                 if (more) {
                     if (!warp_wait(&S.kfull[(n + 1) & 1], ((n + 1) >> 1) & 1, abort, status)) break;
                     tc_fence_after();
                     issue_s(0, n + 1);
                 }
-                if (!warp_wait(&S.pfull[1], n & 1, abort, status)) break;
-                tc_fence_after();
-                issue_pv(1, n);
+                if (!issue_pv(1, n)) break;
                 if (leader) mma_commit(&S.vempty[s]);
                 if (more) {
                     issue_s(1, n + 1);
@@ -897,14 +906,14 @@ __global__ void __launch_bounds__(kFwd3Threads, 1)
                     }
                 }
                 tmem_st32(tmem + lane_off + cS + hc * 32, pk);
+                tmem_st_wait();
+                tc_fence_before();
+                mbar_arrive(&S.pfull[x][hc]);  // this half of P is ready for PV
             }
             float ls[8];
             f2_split(f2_add(lsum2[0], lsum2[2]), ls[0], ls[1]);
             f2_split(f2_add(lsum2[1], lsum2[3]), ls[2], ls[3]);
             l_run += (ls[0] + ls[1]) + (ls[2] + ls[3]);
-            tmem_st_wait();
-            tc_fence_before();
-            mbar_arrive(&S.pfull[x]);
         }
         if (ok && nt > 0 &&
             __all_sync(0xffffffffu, mbar_wait(&S.odone[x], (nt - 1) & 1, abort, status))) {
