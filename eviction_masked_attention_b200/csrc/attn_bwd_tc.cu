@@ -97,6 +97,9 @@ __device__ __forceinline__ void store_row32(__nv_bfloat16 *dst, const uint32_t (
 //   dP^T(n+1) = V dO(n+1)^T
 // (four M=128 N=128 K=128 products): the elementwise phase P^T(n+1) runs while
 // dK(n) and dP^T(n+1) execute, and dS^T(n) while dV(n) and S^T(n+1) execute.
+// P^T and dS^T reach the MMA warp in two halves (the first and second 16 rows
+// of every 32-row part, k-steps 0, 2, 4, 6 and 1, 3, 5, 7 of dV or dK), so each
+// product starts while the elementwise warps still compute its second half.
 // Each product that overwrites a TMEM region is issued after the product that
 // reads it (MMAs run in issue order) and after the elementwise warps reported
 // they had read it.
@@ -120,7 +123,7 @@ struct DkvSmem {
     float dd[kDkvRowStages][128];
     int32_t q0[kDkvRowStages], full_tile[kDkvRowStages];  // tile origin, FULL flag
     uint64_t kv_full, qfull[kDkvQStages], qempty[kDkvQStages], ofull[kDkvOStages], oempty[kDkvOStages],
-        rfull[kDkvRowStages], rempty[kDkvRowStages], st_full, dp_full, p_ready, ds_ready, acc_done, fin;
+        rfull[kDkvRowStages], rempty[kDkvRowStages], st_full, dp_full, p_ready[2], ds_ready[2], acc_done, fin;
     uint32_t tmem_base;
     int abort;
 };
@@ -172,8 +175,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         mbar_init(&S.st_full, 1);
         mbar_init(&S.dp_full, 1);
-        mbar_init(&S.p_ready, kBwdEwThreads);
-        mbar_init(&S.ds_ready, kBwdEwThreads);
+        for (int i = 0; i < 2; ++i) {  // halves h: k-steps h, h+2, h+4, h+6 of dV / dK
+            mbar_init(&S.p_ready[i], kBwdEwThreads);
+            mbar_init(&S.ds_ready[i], kBwdEwThreads);
+        }
         mbar_init(&S.acc_done, 1);
         mbar_init(&S.fin, 1);
         S.abort = 0;
@@ -277,23 +282,40 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 const uint64_t qm = desc_add(qm0, (n % kDkvQStages) * kTile);
                 const uint64_t om = desc_add(om0, (n % kDkvOStages) * kTile);
                 const uint32_t acc = n > 0 ? 1u : 0u;
-                if (!warp_wait(&S.p_ready, n & 1, abort, status)) break;
-                tc_fence_after();
+                // dV(n) in two halves, each issued once the elementwise warps stored the
+                // first (k-steps 0, 2, 4, 6) or second 16 rows of every 32-row part
+                bool okh = true;
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    if (leader)
-                        mma_ts(tmem + cDV, tmem + cST + part_col(kk), desc_add(om, kk * 2048), idMN,
-                               kk > 0 ? 1u : acc);
+                for (int h = 0; h < 2; ++h) {
+                    if (!warp_wait(&S.p_ready[h], n & 1, abort, status)) {
+                        okh = false;
+                        break;
+                    }
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = h; kk < 8; kk += 2)
+                        if (leader)
+                            mma_ts(tmem + cDV, tmem + cST + part_col(kk), desc_add(om, kk * 2048), idMN,
+                                   kk > 0 ? 1u : acc);
+                }
+                if (!okh) break;
                 if (leader) mma_commit(&S.oempty[n % kDkvOStages]);
                 const bool more = n + 1 < nw;
                 if (more && !issue_st(n + 1)) break;
-                if (!warp_wait(&S.ds_ready, n & 1, abort, status)) break;
-                tc_fence_after();
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    if (leader)
-                        mma_ts(tmem + cDK, tmem + cDP + part_col(kk), desc_add(qm, kk * 2048), idMN,
-                               kk > 0 ? 1u : acc);
+                for (int h = 0; h < 2; ++h) {
+                    if (!warp_wait(&S.ds_ready[h], n & 1, abort, status)) {
+                        okh = false;
+                        break;
+                    }
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = h; kk < 8; kk += 2)
+                        if (leader)
+                            mma_ts(tmem + cDK, tmem + cDP + part_col(kk), desc_add(qm, kk * 2048), idMN,
+                                   kk > 0 ? 1u : acc);
+                }
+                if (!okh) break;
                 if (leader) mma_commit(&S.qempty[n % kDkvQStages]);
                 if (more && !issue_dp(n + 1)) break;
             }
@@ -338,68 +360,79 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             // bf16 pairs (the A operand of dV)
             float pf[32];
             {
-                uint32_t r0[32], pk[16];
+                uint32_t r0[32];
                 tmem_ld32(tmem + lane_off + colS, r0);
                 tmem_ld_wait();
                 const float4 *l2v = reinterpret_cast<const float4 *>(S.nl2[s] + 32 * part);
+                const bool masked = __any_sync(0xffffffffu, rlo > 0 || rhi < 32);
+                // in two halves of 16 rows, each handed to the MMA warp as soon as stored
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const float4 lv = l2v[i];
-                    // a quarter of the exponentials on the FMA pipe, the rest on the SFU
-                    float x0, x1, x2, x3;
-                    fma2v(__uint_as_float(r0[4 * i]), __uint_as_float(r0[4 * i + 1]), scale_log2, lv.x, lv.y,
-                          x0, x1);
-                    fma2v(__uint_as_float(r0[4 * i + 2]), __uint_as_float(r0[4 * i + 3]), scale_log2, lv.z,
-                          lv.w, x2, x3);
-                    if (i & 1) {
-                        exp2_fma_x2(x0, x1, pf[4 * i], pf[4 * i + 1]);
-                    } else {
-                        pf[4 * i] = ex2(x0);
-                        pf[4 * i + 1] = ex2(x1);
+                for (int h = 0; h < 2; ++h) {
+#pragma unroll
+                    for (int i = 4 * h; i < 4 * h + 4; ++i) {
+                        const float4 lv = l2v[i];
+                        // a quarter of the exponentials on the FMA pipe, the rest on the SFU
+                        float x0, x1, x2, x3;
+                        fma2v(__uint_as_float(r0[4 * i]), __uint_as_float(r0[4 * i + 1]), scale_log2, lv.x,
+                              lv.y, x0, x1);
+                        fma2v(__uint_as_float(r0[4 * i + 2]), __uint_as_float(r0[4 * i + 3]), scale_log2, lv.z,
+                              lv.w, x2, x3);
+                        if (i & 1) {
+                            exp2_fma_x2(x0, x1, pf[4 * i], pf[4 * i + 1]);
+                        } else {
+                            pf[4 * i] = ex2(x0);
+                            pf[4 * i + 1] = ex2(x1);
+                        }
+                        pf[4 * i + 2] = ex2(x2);
+                        pf[4 * i + 3] = ex2(x3);
                     }
-                    pf[4 * i + 2] = ex2(x2);
-                    pf[4 * i + 3] = ex2(x3);
-                }
-                if (__any_sync(0xffffffffu, rlo > 0 || rhi < 32)) {
+                    if (masked) {
 #pragma unroll
-                    for (int rr = 0; rr < 32; ++rr) pf[rr] = (rr >= rlo && rr < rhi) ? pf[rr] : 0.f;
-                }
+                        for (int rr = 16 * h; rr < 16 * h + 16; ++rr)
+                            pf[rr] = (rr >= rlo && rr < rhi) ? pf[rr] : 0.f;
+                    }
+                    uint32_t pk[8];
 #pragma unroll
-                for (int i = 0; i < 16; ++i) pk[i] = pack_bf16(pf[2 * i], pf[2 * i + 1]);
-                tmem_st16(tmem + lane_off + colS, pk);
+                    for (int i = 0; i < 8; ++i) pk[i] = pack_bf16(pf[16 * h + 2 * i], pf[16 * h + 2 * i + 1]);
+                    tmem_st8(tmem + lane_off + colS + 8 * h, pk);
+                    tmem_st_wait();
+                    tc_fence_before();
+                    mbar_arrive(&S.p_ready[h]);
+                }
             }
-            tmem_st_wait();
-            tc_fence_before();
-            mbar_arrive(&S.p_ready);
             if (!warp_wait(&S.dp_full, ph, abort, status)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            // dS^T = P^T (dP^T - D_t)
+            // dS^T = P^T (dP^T - D_t), in the same two halves
             {
-                uint32_t r0[32], dk2[16];
+                uint32_t r0[32];
                 tmem_ld32(tmem + lane_off + colP, r0);
                 tmem_ld_wait();
                 const float4 *ddv = reinterpret_cast<const float4 *>(S.dd[s] + 32 * part);
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const float4 dv4 = ddv[i];
-                    float d0, d1, d2, d3;
-                    f2_split(f2_mul(f2_make(pf[4 * i], pf[4 * i + 1]),
-                                    f2_sub(f2_make(__uint_as_float(r0[4 * i]), __uint_as_float(r0[4 * i + 1])),
-                                           f2_make(dv4.x, dv4.y))), d0, d1);
-                    f2_split(f2_mul(f2_make(pf[4 * i + 2], pf[4 * i + 3]),
-                                    f2_sub(f2_make(__uint_as_float(r0[4 * i + 2]), __uint_as_float(r0[4 * i + 3])),
-                                           f2_make(dv4.z, dv4.w))), d2, d3);
-                    dk2[2 * i] = pack_bf16(d0, d1);
-                    dk2[2 * i + 1] = pack_bf16(d2, d3);
+                for (int h = 0; h < 2; ++h) {
+                    uint32_t dk2[8];
+#pragma unroll
+                    for (int i = 4 * h; i < 4 * h + 4; ++i) {
+                        const float4 dv4 = ddv[i];
+                        float d0, d1, d2, d3;
+                        f2_split(f2_mul(f2_make(pf[4 * i], pf[4 * i + 1]),
+                                        f2_sub(f2_make(__uint_as_float(r0[4 * i]), __uint_as_float(r0[4 * i + 1])),
+                                               f2_make(dv4.x, dv4.y))), d0, d1);
+                        f2_split(f2_mul(f2_make(pf[4 * i + 2], pf[4 * i + 3]),
+                                        f2_sub(f2_make(__uint_as_float(r0[4 * i + 2]), __uint_as_float(r0[4 * i + 3])),
+                                               f2_make(dv4.z, dv4.w))), d2, d3);
+                        dk2[2 * (i - 4 * h)] = pack_bf16(d0, d1);
+                        dk2[2 * (i - 4 * h) + 1] = pack_bf16(d2, d3);
+                    }
+                    tmem_st8(tmem + lane_off + colP + 8 * h, dk2);
+                    tmem_st_wait();
+                    tc_fence_before();
+                    mbar_arrive(&S.ds_ready[h]);
                 }
-                tmem_st16(tmem + lane_off + colP, dk2);
             }
-            tmem_st_wait();
-            tc_fence_before();
-            mbar_arrive(&S.ds_ready);
             mbar_arrive(&S.rempty[s]);  // done with this item's row data
         }
         // each part writes 32 of the 128 dimensions of dV and dK
