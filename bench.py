@@ -116,11 +116,36 @@ def cpu_baseline_entry(flops: float, secs: float, threads: int, flops_step: floa
             "extrapolated_full_step_s": flops_step / rate}
 
 
+def host_visible_pairs(ev, B: int, N: int) -> int:
+    """Visible (query, key) pairs of the event log: key j is visible from queries j..kappa_j-1,
+    kappa_j the earliest event time covering j (N if none). Host integer arithmetic, used
+    only to describe the workload in the reference arm's config."""
+    total = 0
+    for b in range(B):
+        kap = np.full(N, N, dtype=np.int64)
+        for (s, tau, a, e) in np.asarray(ev).reshape(-1, 4):
+            if s == b:
+                kap[a:e] = np.minimum(kap[a:e], tau)
+        total += int((kap - np.arange(N)).sum())
+    return total
+
+
+def workload_config(cfg, world: int, n_events: int, pairs: float) -> dict:
+    """The bench line's config (both arms)."""
+    return {"workload": f"cfg5 bs1: {cfg.batch}x{cfg.n_tokens} tokens/rank, Hq={cfg.hq}, "
+                        f"Hkv={cfg.hkv}, d={cfg.d}, budget {cfg.budget}, {n_events} events/rank",
+            "global_batch": cfg.batch * world, "seq_len": cfg.n_tokens,
+            "parallelism": f"replicas x{world} (independent traces per rank)",
+            "l2": "inputs larger than L2 (4.3 GB q per rank), no flush",
+            "visible_pair_fraction": pairs / (cfg.batch * cfg.n_tokens * (cfg.n_tokens + 1) / 2)}
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
     cfg = workload_cfg(args.scale)
+    ev = rank_events(cfg, 0)
     budget = 768
     for _ in range(args.warmup):
         oracle_sample(cfg, 256)
@@ -138,7 +163,7 @@ def run_reference(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": "cfg5 bs1 2x131072 Hq64 Hkv8 d128 (bounded oracle sample)"},
+        "config": workload_config(cfg, args.gpus, len(ev), host_visible_pairs(ev, cfg.batch, cfg.n_tokens)),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -772,13 +797,7 @@ def run_ours(args):
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": f"cfg5 bs1: {cfg.batch}x{cfg.n_tokens} tokens/rank, Hq={cfg.hq}, "
-                                   f"Hkv={cfg.hkv}, d={cfg.d}, budget {cfg.budget}, "
-                                   f"{len(step.ev_host)} events/rank",
-                       "global_batch": cfg.batch * world, "seq_len": cfg.n_tokens,
-                       "parallelism": f"replicas x{world} (independent traces per rank)",
-                       "l2": "inputs larger than L2 (4.3 GB q per rank), no flush",
-                       "visible_pair_fraction": P / (cfg.batch * cfg.n_tokens * (cfg.n_tokens + 1) / 2)},
+            "config": workload_config(cfg, world, len(step.ev_host), P),
             "roofline": {"bound": "tensor", "kernel": {"fwd": "k_attn_fwd_tc", "dkdv": "k_attn_dkdv_tc",
                                                        "dq": "k_attn_dq_tc"}[dom],
                          "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,

@@ -80,3 +80,23 @@ def test_cpu_baseline_entry_extrapolates_linearly():
     e = bench.cpu_baseline_entry(2.0e12, 4.0, 16, 1.0e15, "sample")
     assert e["value"] == 0.5 and e["unit"] == "TFLOP/s" and e["kind"] == "oracle" and e["cores"] == 16
     assert e["extrapolated_full_step_s"] == 2000.0
+
+
+def test_host_visible_pairs_counts_the_eventwise_mask():
+    """The reference arm's workload description counts visible pairs on the host;
+    it must equal the pairs of the mask built event by event from the replay rule."""
+    import bench
+    from conftest import dense_mask_eventwise
+    rng = np.random.default_rng(7)
+    for _ in range(20):
+        B, N = int(rng.integers(1, 3)), int(rng.integers(1, 300))
+        ev = []
+        for b in range(B):
+            for _ in range(int(rng.integers(0, 4))):
+                tau = int(rng.integers(1, N + 1))
+                a = int(rng.integers(0, tau))
+                e = int(rng.integers(a + 1, tau + 1))
+                ev.append((b, tau, a, e))
+        ev = np.array(ev, dtype=np.int64).reshape(-1, 4)
+        want = sum(int(dense_mask_eventwise(ev, b, N).sum()) for b in range(B))
+        assert bench.host_visible_pairs(ev, B, N) == want
