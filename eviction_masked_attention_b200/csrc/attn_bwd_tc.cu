@@ -21,7 +21,7 @@
 //   dQ     one CTA per (query tile, head, trace) over the row lists:
 //          S = Q K^T, dP = dO V^T, dS (bit-masked) to TMEM, dQ += dS K.
 // Warp roles: warp 0 TMA, warp 1 TMEM + MMA issue (the whole warp runs the
-// loop, one elected lane issues), warps 2..9 elementwise (thread = TMEM lane).
+// loop, one elected lane issues), warps 2..17 elementwise (thread = TMEM lane).
 #include "common.cuh"
 
 namespace kvs {
