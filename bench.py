@@ -403,7 +403,7 @@ def _durations(rec):
 # 1/16-scale bs1 workload: kernel -> (bytes of that launch, visible pairs x query heads it processed,
 # sha1 prefix of the kernel sources it was taken with). The bench scales it to its own launch by the
 # pairs processed and reports null once the sources have changed.
-TRAFFIC = {"dkdv": (1.779736e9 + 56.255488e6, 27713931 * 64, "04367102d2ee")}
+TRAFFIC = {"dkdv": (1.779736e9 + 56.255488e6, 27713931 * 64, "3fc511ecb941")}
 
 
 def _src_hash(files):
