@@ -273,3 +273,24 @@ def test_full_size_dkdv_long_columns_banded(cid):
         for name, g_, w_ in (("dK", gk, wk), ("dV", gv, wv)):
             rl = rel_l2(g_, w_)
             assert rl is not None and rl <= GRAD_REL_L2, (name, rl)
+
+
+def _bf16_round(x):
+    return torch.from_numpy(np.ascontiguousarray(x)).to(torch.bfloat16).to(torch.float64).numpy()
+
+
+@pytest.mark.parametrize("hq,hkv,with_events", [(4, 2, False), (4, 2, True), (2, 2, False)])
+def test_forward_running_max_rescale(hq, hkv, with_events):
+    """Keys scaled up tile by tile so that each key tile's row maximum exceeds the
+    running maximum by far more than the lazy-rescale threshold: the forward's O
+    rescale (and, for an even group size, the two-half hand-over of P that
+    follows it) runs on every tile. Compared with the oracle as usual."""
+    N = 1024
+    cfg = W.TraceConfig(cid=95, name="rescale", batch=1, n_tokens=N, hq=hq, hkv=hkv, d=128,
+                        theta=1e4, block_size=1, dtype="bf16", prompt=0)
+    q, k, v, do = W.replay_tensors(cfg)
+    f = (1.0 + 4.0 * (np.arange(N) // 128)).reshape(1, N, 1, 1)
+    k = _bf16_round(k * f)
+    ev = (W.random_event_log(np.random.default_rng(11), 1, N, 4, unit=1, max_span=N // 4) if with_events
+          else np.zeros((0, 4), dtype=np.int64))
+    _check_full(cfg, ev, q, k, v, do, BF16_TOL, bwd=False)
