@@ -872,8 +872,10 @@ __global__ void __launch_bounds__(kFwd3Threads, 1)
                 }
             }
             // P = 2^(s*c - m) as bf16 pairs into the first 64 columns of S (all of S is
-            // already in registers). Half of the exponentials run on the FMA pipe
-            // (exp2_fma), half on the special-function unit.
+            // already in registers), all exponentials on the special-function unit: with P
+            // handed over in halves this kernel is bound by the softmax's instruction
+            // latency, and ex2.approx is one instruction per value where the FMA-pipe
+            // cubic takes about five.
             const float nref = m_run == -INFINITY ? 0.f : -m_run;
             uint64_t lsum2[4];  // four f32x2 partial row sums
 #pragma unroll
@@ -890,7 +892,8 @@ __global__ void __launch_bounds__(kFwd3Threads, 1)
                         float x0, x1, x2, x3, p0, p1;
                         fma2(__uint_as_float(rr[j]), __uint_as_float(rr[j + 1]), scale_log2, nref, x0, x1);
                         fma2(__uint_as_float(rr[j + 2]), __uint_as_float(rr[j + 3]), scale_log2, nref, x2, x3);
-                        exp2_fma_x2(x0, x1, p0, p1);
+                        p0 = ex2(x0);
+                        p1 = ex2(x1);
                         float p2 = ex2(x2), p3 = ex2(x3);
                         if (partial) {
                             p0 = ((w >> j) & 1u) ? p0 : 0.f;
