@@ -82,6 +82,9 @@ def rank_events(cfg, rank: int):
 
 # ----------------------------------------------------------------------------- CPU oracle
 
+CPU_SAMPLE_TOKENS = 3584  # about 10-15 s of the oracle on the 16 host cores of a B200 machine
+
+
 def oracle_sample(cfg, budget_tokens: int):
     """The fp64 oracle (as it stands) on a bounded sample of the workload: the
     first ``budget_tokens`` tokens of trace 0 for one kv group (G query heads),
@@ -789,9 +792,10 @@ def run_ours(args):
         dec_gbs = dec_b / (dur["decode"] * 1e-3) / 1e9
         cpu = None
         if not args.no_cpu_baseline and world == 1:
-            f, s, thr = oracle_sample(cfg, 2560)
+            ntok = CPU_SAMPLE_TOKENS
+            f, s, thr = oracle_sample(cfg, ntok)
             cpu = cpu_baseline_entry(f, s, thr, flops_step,
-                                     "first 2560 tokens of trace 0, one kv group (8 query heads), "
+                                     f"first {ntok} tokens of trace 0, one kv group (8 query heads), "
                                      f"fwd + full bwd, {s:.1f} s")
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
