@@ -257,7 +257,9 @@ class Step:
                                   dtype=torch.uint8, device=device)
         self.mask_ws = torch.empty(L.kvs_build_tile_mask_ws_bytes(B, N), dtype=torch.uint8, device=device)
         self.status = torch.zeros(1, dtype=torch.int32, device=device)
+        # counted once here; every step recompiles the log into these buffers
         mask = kvs.kvs_build_tile_mask(self.events, B, N, ws=self.mask_ws)
+        self.mask = mask
         self.pairs = mask.visible_pairs
         self._setup_generation(mask)
 
@@ -322,7 +324,7 @@ class Step:
     # launches of our kernels per step (see each call)
     def launches(self) -> int:
         has_ev = 1 if len(self.ev_host) else 0
-        mask = 2 * (3 + has_ev) + 2        # count call + fill call (+ 2 fill kernels)
+        mask = 3 + has_ev + 2 + 1          # checks, kill times, classes, scans, 2 fills, finish
         return mask + 2 + 1 + 3 + 2 + 1 + 1 + 1 + 1
 
     def run(self, ev_rec=None, bwd_wait=None):
@@ -339,7 +341,7 @@ class Step:
                 ev_rec.setdefault(name, []).append(e)
 
         mark("start")
-        mask = kvs.kvs_build_tile_mask(self.events, B, N, ws=self.mask_ws)
+        mask = kvs.kvs_build_tile_mask_async(self.events, self.mask, ws=self.mask_ws, status=self.status)
         mark("mask")
         kvs.kvs_rope_logical(self.q_raw.view(B * N, Hq, d), self.lpos, cfg.theta, out=self.q.view(B * N, Hq, d))
         kvs.kvs_rope_logical(self.k_raw.view(B * N, Hkv, d), self.lpos, cfg.theta, out=self.k.view(B * N, Hkv, d))
@@ -455,7 +457,7 @@ def _attn_config(cid: int, dev, peaks, bwd: bool, scale: int = 1):
     q, k, v, do = W.replay_tensors_device(cfg, device=dev, with_grad=bwd)
     mask_ws = torch.empty(kvs.lib().kvs_build_tile_mask_ws_bytes(B, N), dtype=torch.uint8, device=dev)
     mask = kvs.kvs_build_tile_mask(ev, B, N, ws=mask_ws)
-    t_mask = _time_ms(lambda: kvs.kvs_build_tile_mask(ev, B, N, ws=mask_ws), 5)
+    t_mask = _time_ms(lambda: kvs.kvs_build_tile_mask_async(ev, mask, ws=mask_ws), 5)
     P = float(mask.visible_pairs)
     o, lse, o_lo = torch.empty_like(q), torch.empty((B, Hq, N), dtype=torch.float32, device=dev), torch.empty_like(q)
     st = torch.zeros(1, dtype=torch.int32, device=dev)

@@ -33,6 +33,7 @@ EXPORTED = (
     "kvs_rope_logical", "kvs_paged_decode_ws_bytes", "kvs_paged_decode_attn",
     "kvs_masked_attn_fwd", "kvs_masked_attn_bwd_ws_bytes", "kvs_masked_attn_bwd",
     "kvs_status_str", "kvs_version", "kvs_last_cuda_error", "kvs_paged_decode_attn_static",
+    "kvs_build_tile_mask_async",
 )
 
 
@@ -72,6 +73,7 @@ def lib() -> C.CDLL:
         L.kvs_build_tile_mask_ws_bytes.restype = sz
         L.kvs_build_tile_mask.argtypes = [vp, i32, i32, i32, C.POINTER(_TileMaskC), C.POINTER(_SizesC),
                                           vp, sz, vp]
+        L.kvs_build_tile_mask_async.argtypes = [vp, i32, i32, i32, C.POINTER(_TileMaskC), vp, vp, sz, vp, vp]
         L.kvs_compact_block_table.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, vp, i32, vp, vp, vp, vp]
         L.kvs_rope_logical.argtypes = [vp, i64, vp, vp, i32, i32, i32, f64, i32, vp, i32, i32, vp, i64,
                                        vp, i32, vp, vp]
@@ -91,7 +93,7 @@ def lib() -> C.CDLL:
         L.kvs_status_str.restype = C.c_char_p
         L.kvs_version.restype = i32
         L.kvs_last_cuda_error.restype = C.c_char_p
-        for r in ("kvs_build_tile_mask", "kvs_compact_block_table", "kvs_rope_logical",
+        for r in ("kvs_build_tile_mask", "kvs_build_tile_mask_async", "kvs_compact_block_table", "kvs_rope_logical",
                   "kvs_paged_decode_attn", "kvs_paged_decode_attn_static", "kvs_masked_attn_fwd",
                   "kvs_masked_attn_bwd"):
             getattr(L, r).restype = i32
@@ -196,6 +198,34 @@ def kvs_build_tile_mask(events: torch.Tensor, B: int, N: int, ws: Optional[torch
     _check(L.kvs_build_tile_mask(evp, n_ev, B, N, C.byref(m2), C.byref(sizes), _p(ws), wsb, _stream()),
            "kvs_build_tile_mask(fill)")
     return out
+
+
+def kvs_build_tile_mask_async(events: torch.Tensor, mask: TileMask, ws: Optional[torch.Tensor] = None,
+                              sizes: Optional[torch.Tensor] = None,
+                              status: Optional[torch.Tensor] = None) -> TileMask:
+    """Recompile an event log into the buffers of ``mask`` (same B and N; list
+    capacities are the buffers' sizes) with one asynchronous library call: no
+    host round trip. ``sizes`` (int64 [3]: nnz, n_partial, visible pairs) and
+    ``status`` (int32 [1], first error wins) are device tensors or None; on an
+    event-log error or lists over capacity the status is set and the mask reads
+    as empty. ``mask.nnz`` etc. keep the values of the build that made it."""
+    if events.numel() == 0:
+        events = torch.zeros((0, 4), dtype=torch.int32, device=mask.kappa.device)
+    _dev(events)
+    assert events.dtype == torch.int32 and events.shape[-1] == 4
+    L = lib()
+    wsb = L.kvs_build_tile_mask_ws_bytes(mask.B, mask.N)
+    if ws is None or ws.numel() < wsb:
+        ws = torch.empty(wsb, dtype=torch.uint8, device=mask.kappa.device)
+    if sizes is not None:
+        assert sizes.dtype == torch.int64 and sizes.numel() >= 3
+    m = mask.c_struct()
+    n_ev = events.shape[0]
+    _check(L.kvs_build_tile_mask_async(_p(events) if n_ev else None, n_ev, mask.B, mask.N, C.byref(m),
+                                       _p(sizes) if sizes is not None else None, _p(ws), wsb,
+                                       _p(status) if status is not None else None, _stream()),
+           "kvs_build_tile_mask_async")
+    return mask
 
 
 # ------------------------------------------------------------------------------ compaction

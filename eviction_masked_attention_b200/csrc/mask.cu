@@ -210,10 +210,13 @@ __global__ void k_scan3(const int32_t *in0, int32_t *out0, const int32_t *in1, i
 __global__ void k_fill_rows(const int32_t *__restrict__ kappa, const uint8_t *__restrict__ cls,
                             int32_t B, int32_t N, int32_t T, const int32_t *__restrict__ row_ptr,
                             const int32_t *__restrict__ row_poff, int32_t *row_col,
-                            int32_t *row_pidx, int32_t *tile_pidx, uint32_t *bits) {
+                            int32_t *row_pidx, int32_t *tile_pidx, uint32_t *bits, int64_t nnz_cap,
+                            int64_t partial_cap) {
     const int lane = threadIdx.x & 31;
     const int32_t row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (row >= B * T) return;
+    // lists that do not fit are not written at all (the asynchronous build has no host check)
+    if (row_ptr[B * T] > nnz_cap || row_poff[B * T] > partial_cap) return;
     const int32_t b = row / T, qi = row % T, q0 = qi * 128;
     const int32_t *kap = kappa + (int64_t)b * N;
     const uint8_t *crow = cls + (int64_t)row * T;
@@ -271,10 +274,12 @@ __global__ void k_fill_rows(const int32_t *__restrict__ kappa, const uint8_t *__
 __global__ void k_fill_cols(const uint8_t *__restrict__ cls, int32_t B, int32_t T,
                             const int32_t *__restrict__ col_ptr,
                             const int32_t *__restrict__ tile_pidx, int32_t *col_row,
-                            int32_t *col_pidx) {
+                            int32_t *col_pidx, const int32_t *__restrict__ row_poff, int64_t nnz_cap,
+                            int64_t partial_cap) {
     const int lane = threadIdx.x & 31;
     const int32_t col = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (col >= B * T) return;
+    if (col_ptr[B * T] > nnz_cap || row_poff[B * T] > partial_cap) return;
     const int32_t b = col / T, kj = col % T;
     int32_t e = col_ptr[col];
     const unsigned lt = (1u << lane) - 1u;
@@ -292,6 +297,33 @@ __global__ void k_fill_cols(const uint8_t *__restrict__ cls, int32_t B, int32_t 
     }
 }
 
+// Last step of the asynchronous build: report the sizes, and on an event-log
+// error or lists over capacity record the status and leave the mask empty
+// (every row and column list of length zero), so that an attention call that
+// runs on it anyway reads nothing it should not.
+__global__ void k_mask_finish(int32_t *row_ptr, int32_t *col_ptr, const int32_t *__restrict__ row_poff,
+                              const int32_t *__restrict__ ev_status,
+                              const unsigned long long *__restrict__ pairs, int32_t BT, int64_t nnz_cap,
+                              int64_t partial_cap, int64_t *sizes, int32_t *status) {
+    const int32_t nnz = row_ptr[BT], np = row_poff[BT], est = *ev_status;
+    const bool over = nnz > nnz_cap || np > partial_cap;
+    __syncthreads();  // every thread has read the totals before any clears them
+    if (threadIdx.x == 0) {
+        if (sizes) {
+            sizes[0] = nnz;
+            sizes[1] = np;
+            sizes[2] = (int64_t)*pairs;
+        }
+        if (est) set_status(status, est);
+        else if (over) set_status(status, KVS_ERR_CAPACITY);
+    }
+    if (est || over)
+        for (int32_t i = threadIdx.x; i <= BT; i += blockDim.x) {
+            row_ptr[i] = 0;
+            col_ptr[i] = 0;
+        }
+}
+
 }  // namespace kvs
 
 using namespace kvs;
@@ -301,21 +333,27 @@ extern "C" size_t kvs_build_tile_mask_ws_bytes(int32_t B, int32_t N) {
     return mask_ws_layout(B, N, nullptr, nullptr);
 }
 
-extern "C" kvs_status kvs_build_tile_mask(const kvs_evict_range *ev, int32_t n_ev, int32_t B,
-                                          int32_t N, kvs_tile_mask *m, kvs_mask_sizes *sizes,
-                                          void *ws, size_t ws_bytes, kvs_stream_t stream) {
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    if (!m || !sizes || B <= 0 || N <= 0 || n_ev < 0 || (n_ev > 0 && !ev)) return KVS_ERR_INVALID_ARG;
+namespace {
+
+// Host checks shared by both builds; fills *w from ws.
+kvs_status mask_args(const kvs_evict_range *ev, int32_t n_ev, int32_t B, int32_t N, kvs_tile_mask *m,
+                     void *ws, size_t ws_bytes, MaskWs *w) {
+    if (!m || B <= 0 || N <= 0 || n_ev < 0 || (n_ev > 0 && !ev)) return KVS_ERR_INVALID_ARG;
     if (m->B != B || m->N != N) return KVS_ERR_INVALID_ARG;
     const int64_t T64 = (N + 127) / 128;
     if ((int64_t)B * T64 * T64 >= (1ll << 31)) return KVS_ERR_CAPACITY;
-    const int32_t T = (int32_t)T64;
-    m->T = T;
+    m->T = (int32_t)T64;
     if (!m->kappa || !m->cls || !m->row_ptr || !m->col_ptr) return KVS_ERR_INVALID_ARG;
     if (!ws || ws_bytes < kvs_build_tile_mask_ws_bytes(B, N)) return KVS_ERR_CAPACITY;
-    MaskWs w;
-    mask_ws_layout(B, N, &w, (char *)ws);
-    const int32_t BT = B * T;
+    mask_ws_layout(B, N, w, (char *)ws);
+    return KVS_OK;
+}
+
+// Event checks, kill times, tile classes and the three scans (row offsets,
+// partial offsets, column offsets).
+kvs_status mask_count(const kvs_evict_range *ev, int32_t n_ev, int32_t B, int32_t N,
+                      const kvs_tile_mask *m, const MaskWs &w, cudaStream_t s) {
+    const int32_t T = m->T, BT = B * T;
     cudaError_t ce;
     if ((ce = cudaMemsetAsync(w.col_cnt, 0, sizeof(int32_t) * BT, s)) != cudaSuccess ||
         (ce = cudaMemsetAsync(w.status, 0, sizeof(int32_t) * 4, s)) != cudaSuccess ||
@@ -327,7 +365,37 @@ extern "C" kvs_status kvs_build_tile_mask(const kvs_evict_range *ev, int32_t n_e
     k_classify<<<BT, 256, 0, s>>>(m->kappa, B, N, T, m->cls, w.row_nnz, w.row_npart, w.col_cnt);
     k_scan3<<<3, 1024, 0, s>>>(w.row_nnz, m->row_ptr, w.row_npart, w.row_poff, w.col_cnt,
                                m->col_ptr, BT);
-    if ((ce = cudaGetLastError()) != cudaSuccess) return cuda_status(ce);
+    return (ce = cudaGetLastError()) != cudaSuccess ? cuda_status(ce) : KVS_OK;
+}
+
+// Row and column lists and the bit rows of partial tiles, each kernel skipping
+// all writes when the totals exceed the capacities.
+kvs_status mask_fill(int32_t B, int32_t N, const kvs_tile_mask *m, const MaskWs &w, cudaStream_t s) {
+    const int32_t T = m->T, BT = B * T;
+    const int rows_per_cta = 8;
+    k_fill_rows<<<(BT + rows_per_cta - 1) / rows_per_cta, 32 * rows_per_cta, 0, s>>>(
+        m->kappa, m->cls, B, N, T, m->row_ptr, w.row_poff, m->row_col, m->row_pidx, w.tile_pidx,
+        m->bits, m->nnz_cap, m->partial_cap);
+    k_fill_cols<<<(BT + rows_per_cta - 1) / rows_per_cta, 32 * rows_per_cta, 0, s>>>(
+        m->cls, B, T, m->col_ptr, w.tile_pidx, m->col_row, m->col_pidx, w.row_poff, m->nnz_cap,
+        m->partial_cap);
+    cudaError_t ce;
+    return (ce = cudaGetLastError()) != cudaSuccess ? cuda_status(ce) : KVS_OK;
+}
+
+}  // namespace
+
+extern "C" kvs_status kvs_build_tile_mask(const kvs_evict_range *ev, int32_t n_ev, int32_t B,
+                                          int32_t N, kvs_tile_mask *m, kvs_mask_sizes *sizes,
+                                          void *ws, size_t ws_bytes, kvs_stream_t stream) {
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (!sizes) return KVS_ERR_INVALID_ARG;
+    MaskWs w;
+    kvs_status st = mask_args(ev, n_ev, B, N, m, ws, ws_bytes, &w);
+    if (st != KVS_OK) return st;
+    if ((st = mask_count(ev, n_ev, B, N, m, w, s)) != KVS_OK) return st;
+    const int32_t BT = B * m->T;
+    cudaError_t ce;
     int32_t h_nnz = 0, h_np = 0, h_st = 0;
     unsigned long long h_pairs = 0;
     if ((ce = cudaMemcpyAsync(&h_nnz, m->row_ptr + BT, 4, cudaMemcpyDeviceToHost, s)) != cudaSuccess ||
@@ -344,12 +412,24 @@ extern "C" kvs_status kvs_build_tile_mask(const kvs_evict_range *ev, int32_t n_e
     if (!m->row_pidx || !m->col_row || !m->col_pidx || (h_np > 0 && !m->bits))
         return KVS_ERR_INVALID_ARG;
     if (h_nnz > m->nnz_cap || h_np > m->partial_cap) return KVS_ERR_CAPACITY;
-    const int rows_per_cta = 8;
-    k_fill_rows<<<(BT + rows_per_cta - 1) / rows_per_cta, 32 * rows_per_cta, 0, s>>>(
-        m->kappa, m->cls, B, N, T, m->row_ptr, w.row_poff, m->row_col, m->row_pidx, w.tile_pidx,
-        m->bits);
-    k_fill_cols<<<(BT + rows_per_cta - 1) / rows_per_cta, 32 * rows_per_cta, 0, s>>>(
-        m->cls, B, T, m->col_ptr, w.tile_pidx, m->col_row, m->col_pidx);
-    if ((ce = cudaGetLastError()) != cudaSuccess) return cuda_status(ce);
-    return KVS_OK;
+    return mask_fill(B, N, m, w, s);
+}
+
+extern "C" kvs_status kvs_build_tile_mask_async(const kvs_evict_range *ev, int32_t n_ev, int32_t B,
+                                                int32_t N, kvs_tile_mask *m, int64_t *dev_sizes,
+                                                void *ws, size_t ws_bytes, int32_t *dev_status,
+                                                kvs_stream_t stream) {
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    MaskWs w;
+    kvs_status st = mask_args(ev, n_ev, B, N, m, ws, ws_bytes, &w);
+    if (st != KVS_OK) return st;
+    if (!m->row_col || !m->row_pidx || !m->col_row || !m->col_pidx || m->nnz_cap < 0 ||
+        m->partial_cap < 0 || (m->partial_cap > 0 && !m->bits))
+        return KVS_ERR_INVALID_ARG;
+    if ((st = mask_count(ev, n_ev, B, N, m, w, s)) != KVS_OK) return st;
+    if ((st = mask_fill(B, N, m, w, s)) != KVS_OK) return st;
+    k_mask_finish<<<1, 256, 0, s>>>(m->row_ptr, m->col_ptr, w.row_poff, w.status, w.pairs, B * m->T,
+                                    m->nnz_cap, m->partial_cap, dev_sizes, dev_status);
+    cudaError_t ce;
+    return (ce = cudaGetLastError()) != cudaSuccess ? cuda_status(ce) : KVS_OK;
 }

@@ -22,7 +22,8 @@
  *    library's device image, and it caches that array's device address per
  *    device and CUDA context (see its comment).
  *  - Every call is asynchronous on `stream`, except kvs_build_tile_mask, which
- *    synchronises `stream` once to learn the sizes of its outputs.
+ *    synchronises `stream` once to learn the sizes of its outputs
+ *    (kvs_build_tile_mask_async is its asynchronous form).
  *  - Errors the host can see (NULL or misaligned pointers, bad sizes,
  *    unsupported dtype/head size) are returned at once and nothing is
  *    launched. Errors that depend on device data are written to `*dev_status`
@@ -123,6 +124,26 @@ size_t kvs_build_tile_mask_ws_bytes(int32_t B, int32_t N);
 kvs_status kvs_build_tile_mask(const kvs_evict_range *ev, int32_t n_ev, int32_t B, int32_t N,
                                kvs_tile_mask *m, kvs_mask_sizes *sizes, void *ws, size_t ws_bytes,
                                kvs_stream_t stream);
+
+/*
+ * The same compilation without the host round trip, for a training loop that
+ * keeps the mask buffers from step to step: nothing is read back and `stream`
+ * is never synchronised, so the call neither stalls the host nor waits behind
+ * other device-to-host copies.
+ *   m          as above, with every list pointer set (bits may be NULL only
+ *              when partial_cap == 0) and nnz_cap / partial_cap the capacity
+ *              of the buffers, e.g. from a counting call on the same log or a
+ *              bound the caller derives.
+ *   dev_sizes  device int64 [3] or NULL: nnz, n_partial, visible_pairs.
+ *   dev_status device int32 (first error wins) or NULL.
+ * Event-log errors (as above) and lists over capacity (KVS_ERR_CAPACITY) are
+ * written to *dev_status; the lists are then not written and every row_ptr and
+ * col_ptr entry is set to 0, so the mask reads as empty. Host-visible argument
+ * errors are returned at once and nothing is launched.
+ */
+kvs_status kvs_build_tile_mask_async(const kvs_evict_range *ev, int32_t n_ev, int32_t B, int32_t N,
+                                     kvs_tile_mask *m, int64_t *dev_sizes, void *ws, size_t ws_bytes,
+                                     int32_t *dev_status, kvs_stream_t stream);
 
 /*
  * Block-table compaction ([T] second fix: only whole blocks leave the cache,

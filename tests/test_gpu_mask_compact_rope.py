@@ -67,6 +67,102 @@ def test_mask_event_errors(bad, code):
     assert e.value.code == code
 
 
+# ------------------------------------------------- mask, asynchronous build
+
+_SENT = -7
+
+
+def _mask_buffers(B, N, nnz_cap, part_cap, extra=64):
+    """A TileMask whose list buffers hold nnz_cap / part_cap entries (views of
+    larger sentinel-filled stores, so writes past the capacity would stay in
+    allocated memory and show up as changed sentinels)."""
+    T = (N + 127) // 128
+    i32 = dict(dtype=torch.int32, device="cuda")
+    stores = [torch.full((max(nnz_cap, 1) + extra,), _SENT, **i32) for _ in range(4)]
+    bstore = torch.full(((max(part_cap, 1) + 1) * 512,), _SENT, **i32)
+    lists = [st[:max(nnz_cap, 1)] for st in stores]
+    bits = bstore[:max(part_cap, 1) * 512].view(-1, 128, 4)
+    m = kvs.TileMask(B, N, T, torch.full((B, N), _SENT, **i32),
+                     torch.zeros((B, T, T), dtype=torch.uint8, device="cuda"),
+                     torch.full((B * T + 1,), _SENT, **i32), lists[0], lists[1],
+                     torch.full((B * T + 1,), _SENT, **i32), lists[2], lists[3], bits, 0, 0, 0)
+    return m, stores, bstore
+
+
+def _async_build(ev, m):
+    sizes = torch.zeros(3, dtype=torch.int64, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    kvs.kvs_build_tile_mask_async(events_dev(ev), m, sizes=sizes, status=status)
+    torch.cuda.synchronize()
+    return [int(x) for x in sizes.cpu()], int(status.item())
+
+
+@pytest.mark.parametrize("cid,div", [(1, 1), (2, 8), (5, 16)])
+def test_mask_async_configs(cid, div):
+    """The host-round-trip-free build, with capacities from the oracle's counts,
+    equals the oracle bit for bit (lists, bits and the device-reported sizes)."""
+    cfg = W.scaled(W.CONFIGS[cid], div)
+    ev = W.make_event_log(cfg)
+    B, N = cfg.batch, cfg.n_tokens
+    om = oracle.tile_mask(oracle.kappa(ev, B, N))
+    m, _, _ = _mask_buffers(B, N, om["nnz"], om["n_partial"])
+    (nnz, npart, pairs), st = _async_build(ev, m)
+    assert st == 0
+    m.nnz, m.n_partial, m.visible_pairs = nnz, npart, pairs
+    compare_mask(m, ev, B, N)
+
+
+@pytest.mark.parametrize("N,seed", [(300, 1), (1000, 2), (129, 4)])
+def test_mask_async_reuses_buffers(N, seed):
+    """A training loop recompiles each step's log into the buffers of an earlier
+    build: a second, different log into the same buffers gives its own mask."""
+    rng = np.random.default_rng(seed)
+    ev1 = W.random_event_log(rng, 3, N, 12, unit=1, max_span=max(1, N // 4))
+    ev2 = W.random_event_log(rng, 3, N, 6, unit=1, max_span=max(1, N // 8))
+    gm = kvs.kvs_build_tile_mask(events_dev(ev1), 3, N)
+    om2 = oracle.tile_mask(oracle.kappa(ev2, 3, N))
+    if om2["nnz"] > gm.row_col.numel() or om2["n_partial"] > gm.bits.shape[0]:
+        gm, _, _ = _mask_buffers(3, N, om2["nnz"], om2["n_partial"])
+    (nnz, npart, pairs), st = _async_build(ev2, gm)
+    assert st == 0
+    gm.nnz, gm.n_partial, gm.visible_pairs = nnz, npart, pairs
+    compare_mask(gm, ev2, 3, N)
+
+
+@pytest.mark.parametrize("short", ["nnz", "partial"])
+def test_mask_async_over_capacity(short):
+    """Lists that do not fit: KVS_ERR_CAPACITY in the status word, the sizes
+    still reported, no list entry or bit row written, and every row/column
+    offset zero (the mask reads as empty)."""
+    rng = np.random.default_rng(11)
+    B, N = 3, 1000
+    ev = W.random_event_log(rng, B, N, 12, unit=1, max_span=N // 4)
+    om = oracle.tile_mask(oracle.kappa(ev, B, N))
+    assert om["nnz"] >= 2 and om["n_partial"] >= 2
+    nc = om["nnz"] - (1 if short == "nnz" else 0)
+    pc = om["n_partial"] - (1 if short == "partial" else 0)
+    m, stores, bstore = _mask_buffers(B, N, nc, pc)
+    (nnz, npart, pairs), st = _async_build(ev, m)
+    assert st == kvs.KVS_ERR_CAPACITY
+    assert (nnz, npart) == (om["nnz"], om["n_partial"])
+    assert pairs == oracle.visible_pairs(oracle.kappa(ev, B, N))
+    assert not m.row_ptr.any().item() and not m.col_ptr.any().item()
+    for t in stores + [bstore]:
+        assert bool((t == _SENT).all().item())
+
+
+@pytest.mark.parametrize("bad,code", [
+    ([[0, 100, 10, 20], [0, 50, 0, 10]], kvs.KVS_ERR_EVENT_ORDER),
+    ([[5, 100, 10, 20]], kvs.KVS_ERR_INVALID_ARG),
+])
+def test_mask_async_event_errors(bad, code):
+    """Event-log errors land in the status word and leave the mask empty."""
+    m, _, _ = _mask_buffers(2, 256, 8, 8)
+    _, st = _async_build(bad, m)
+    assert st == code
+    assert not m.row_ptr.any().item() and not m.col_ptr.any().item()
+
+
 # ------------------------------------------------------------------ compaction
 
 def _compact_gpu(st, events):
