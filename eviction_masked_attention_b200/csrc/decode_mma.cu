@@ -63,8 +63,17 @@ __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], 
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+// K/V rows are read once per call: they enter L2 as the first lines to evict, so the
+// stream does not push out what the kernels before the decode left there (a step's
+// last kernels leave L2 full of lines still to be written back)
+__device__ __forceinline__ uint64_t l2_evict_first() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint64_t pol) {
+    asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "l"(pol)
+                 : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() {
     asm volatile("cp.async.commit_group;" ::: "memory");
@@ -98,6 +107,7 @@ __global__ void __launch_bounds__(kDmThreads, 3)
     if (rg.x0 >= rg.x1) return;
     const int64_t blk_stride = (int64_t)Hkv * bs * D;
     const int piece = lane & 15, par = lane >> 4;
+    const uint64_t pol = l2_evict_first();
     const int g = lane >> 2, t4 = lane & 3;
     // chunks of one sub-piece: its ids (at most (chunks * 16 - 1) / bs + 2 of them)
     // must fit the kDmMaxTps + 16 staged slots
@@ -173,8 +183,8 @@ __global__ void __launch_bounds__(kDmThreads, 3)
                         for (int j = 0; j < 8; ++j) {
                             const int e = par + 2 * j;
                             if (e < nv && id >= 0) {
-                                cp_async16(kd + e * kDmRow, kc + base + e * D);
-                                cp_async16(vd + e * kDmRow, vc + base + e * D);
+                                cp_async16(kd + e * kDmRow, kc + base + e * D, pol);
+                                cp_async16(vd + e * kDmRow, vc + base + e * D, pol);
                             }
                         }
                     } else {
@@ -188,8 +198,8 @@ __global__ void __launch_bounds__(kDmThreads, 3)
                                                             : (int64_t)id * blk_stride + head_off +
                                                                   (int64_t)(t % bs) * D + piece * 8;
                                 if (id >= 0) {
-                                    cp_async16(kd + e * kDmRow, kc + off);
-                                    cp_async16(vd + e * kDmRow, vc + off);
+                                    cp_async16(kd + e * kDmRow, kc + off, pol);
+                                    cp_async16(vd + e * kDmRow, vc + off, pol);
                                 }
                             }
                         }
