@@ -325,7 +325,9 @@ class Step:
     def launches(self) -> int:
         has_ev = 1 if len(self.ev_host) else 0
         mask = 3 + has_ev + 2 + 1          # checks, kill times, classes, scans, 2 fills, finish
-        return mask + 2 + 1 + 3 + 2 + 1 + 1 + 1 + 1
+        # RoPE of q and k, forward, prep + dK/dV + dQ, inverse RoPE of dq and dk, compaction,
+        # RoPE + scatter of the new key and value, RoPE of the new query, decode split + merge
+        return mask + 2 + 1 + 3 + 2 + 1 + 1 + 1 + 2
 
     def run(self, ev_rec=None, bwd_wait=None):
         """One step; if ev_rec is a dict, records CUDA events around each call. With
