@@ -56,6 +56,17 @@ def test_host_side_argument_errors(built):
                                    None, None, 0, None, None) == kvs.KVS_ERR_INVALID_ARG
     assert L.kvs_paged_decode_attn(None, None, None, None, None, 1, 8, 1, 128, 16, 2**27, 8, 1.0,
                                    kvs.KVS_BF16, None, None, 0, None, None) == kvs.KVS_ERR_CAPACITY
+    # the asynchronous mask build checks its arguments on the host and launches nothing
+    # when they are bad: no mask struct, a B/N mismatch, or list buffers missing
+    assert L.kvs_build_tile_mask_async(None, 0, 1, 100, None, None, None, 0, None,
+                                       None) == kvs.KVS_ERR_INVALID_ARG
+    mm = kvs._TileMaskC()
+    mm.B, mm.N = 2, 100
+    assert L.kvs_build_tile_mask_async(None, 0, 1, 100, ctypes.byref(mm), None, None, 0, None,
+                                       None) == kvs.KVS_ERR_INVALID_ARG
+    mm.B = 1
+    assert L.kvs_build_tile_mask_async(None, 0, 1, 100, ctypes.byref(mm), None, None, 0, None,
+                                       None) == kvs.KVS_ERR_INVALID_ARG
     m = kvs._TileMaskC()
     m.B, m.N, m.T = 1, 100, 1
     assert L.kvs_masked_attn_fwd(None, None, None, ctypes.byref(m), 1, 100, 4, 1, 96, 1.0, kvs.KVS_BF16,
