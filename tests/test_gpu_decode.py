@@ -85,6 +85,83 @@ def test_decode_bs1_bf16_scaled():
     assert_close(got, want, BF16_TOL, "bs1 decode")
 
 
+def test_decode_bs1_full_size():
+    """The bs1 trace workload's decode at full size, in the launch configuration the
+    step times: two traces of 131 072 positions, 1-token blocks at random slots, each
+    trace's table right before its last event compacted through the library, the new
+    token roped and appended at its logical position, then one decode call (a wave of
+    split CTAs and the merge). The compacted tables must hold exactly the keys the
+    oracle's kill times keep, and every query head must match the oracle's replay
+    row at that position."""
+    cfg = W.CONFIGS[5]
+    B, N, Hq, Hkv, d = cfg.batch, cfg.n_tokens, cfg.hq, cfg.hkv, cfg.d
+    G = Hq // Hkv
+    ev = W.make_event_log(cfg)
+    kap = oracle.kappa(ev, B, N)
+    q_raw, k_raw, v, _ = W.replay_tensors_device(cfg, device="cuda", with_grad=False)
+    pool = B * N + B
+    perm = np.random.default_rng(77).permutation(pool).astype(np.int64)
+    kc = torch.zeros((pool, Hkv, 1, d), dtype=torch.bfloat16, device="cuda")
+    vc = torch.zeros_like(kc)
+    lpos = torch.arange(N, dtype=torch.int32, device="cuda")
+    taus, tables, lposs = [], [], []
+    for b in range(B):
+        tau = int(ev[ev[:, 0] == b, 1].max())
+        j = np.arange(tau)
+        live = j[kap[b, :tau] >= tau]  # alive right before the event at tau
+        taus.append(tau)
+        tables.append(perm[b * N + live].astype(np.int32))
+        lposs.append(live.astype(np.int32))
+        kvs.kvs_rope_logical(k_raw[b], lpos, cfg.theta, out=kc, out_slot=dev(perm[b * N:(b + 1) * N]),
+                             block_size=1, v=v[b], v_out=vc)
+    M = max(len(t) for t in tables) + 1
+    bt = np.full((B, M), -1, np.int32)
+    bl = np.full((B, M), -1, np.int32)
+    for b in range(B):
+        bt[b, :len(tables[b])] = tables[b]
+        bl[b, :len(lposs[b])] = lposs[b]
+    nb = np.array([len(t) for t in tables], np.int32)
+    dbt, dbl, dnb, dnt = dev(bt), dev(bl), dev(nb), dev(nb)
+    last = np.concatenate([ev[(ev[:, 0] == b) & (ev[:, 1] == taus[b])] for b in range(B)])
+    _, _, status = kvs.kvs_compact_block_table(dbt, dbl, dnb, dnt, 1, pool, events_dev(last))
+    # the new token of trace b: logical position tau_b, physical slot perm[B N + b]
+    tl = dev(np.array(taus, np.int32))
+    rows = torch.from_numpy(np.array([b * N + taus[b] for b in range(B)])).cuda()
+    qn = q_raw.view(B * N, Hq, d).index_select(0, rows)
+    kn = k_raw.view(B * N, Hkv, d).index_select(0, rows).contiguous()
+    vn = v.view(B * N, Hkv, d).index_select(0, rows).contiguous()
+    new_slot = perm[B * N:B * N + B]
+    kvs.kvs_rope_logical(kn, tl, cfg.theta, out=kc, out_slot=dev(new_slot), block_size=1, v=vn, v_out=vc)
+    qr = kvs.kvs_rope_logical(qn, tl, cfg.theta)
+    # the oracle's inputs (raw rows up to tau) move to the host; the decode then runs
+    # with only the caches and tables on the device
+    raw = [(host(q_raw[b, taus[b]]), host(k_raw[b, :taus[b] + 1]), host(v[b, :taus[b] + 1])) for b in range(B)]
+    del q_raw, k_raw, v, qn, kn, vn
+    torch.cuda.empty_cache()
+    nb_after = dnb.cpu().numpy()
+    dbt[torch.arange(B, device="cuda"), torch.from_numpy(nb_after.astype(np.int64)).cuda()] = \
+        dev(new_slot.astype(np.int32))
+    dnt += 1
+    o = host(kvs.kvs_paged_decode_attn(qr, kc, vc, dbt, dnt, 1, cfg.scale, status=status))
+    assert int(status.item()) == 0
+    got_bt = dbt.cpu().numpy()
+    for b in range(B):
+        tau = taus[b]
+        keep = np.arange(tau)[kap[b, :tau] > tau]  # kept by the event at tau
+        assert nb_after[b] == len(keep)
+        assert np.array_equal(got_bt[b, :nb_after[b]], perm[b * N + keep].astype(np.int32))
+        # oracle: raw keys and values up to tau, rotated in fp64, replay row tau
+        qh, kh, vv = raw[b]
+        kr = oracle.rope(kh, np.arange(tau + 1), cfg.theta)
+        qo = oracle.rope(qh[None], [tau], cfg.theta)[0]
+        want = np.empty((Hq, d))
+        for h in range(Hq):
+            r, _ = oracle.attn_rows(qo[h][None], [tau], kr[:, h // G], vv[:, h // G], kap[b, :tau + 1],
+                                    cfg.scale)
+            want[h] = r[0]
+        assert_close(o[b], want, BF16_TOL, f"bs1 full-size decode seq {b}")
+
+
 def _paged_step(div):
     """One generation step of the paged workload: compaction, RoPE + append of the
     new token at its logical position, decode. Returns what the oracle needs."""
