@@ -475,7 +475,9 @@ def _attn_config(cid: int, dev, peaks, bwd: bool, scale: int = 1):
         bw = lambda: kvs.kvs_masked_attn_bwd(q, k, v, o, do, lse, mask, cfg.scale, dq=dq, dk=dk, dv=dv, ws=ws,
                                              status=st, o_lo=o_lo)
         t_bwd = _time_ms(bw, 5)
+        # 10 d per pair counts the backward's five products (S recomputed); 8 d leaves the recompute out
         out.update({"bwd_ms": t_bwd, "bwd_tflops": 10 * d * P * Hq / (t_bwd * 1e-3) / 1e12,
+                    "bwd_tflops_8d": 8 * d * P * Hq / (t_bwd * 1e-3) / 1e12,
                     "fwd_bwd_tflops": 14 * d * P * Hq / ((t_fwd + t_bwd) * 1e-3) / 1e12})
         tf = out["fwd_bwd_tflops"]
     else:
