@@ -138,8 +138,9 @@ kvs_status kvs_build_tile_mask(const kvs_evict_range *ev, int32_t n_ev, int32_t 
  *   dev_status device int32 (first error wins) or NULL.
  * Event-log errors (as above) and lists over capacity (KVS_ERR_CAPACITY) are
  * written to *dev_status; the lists are then not written and every row_ptr and
- * col_ptr entry is set to 0, so the mask reads as empty. Host-visible argument
- * errors are returned at once and nothing is launched.
+ * col_ptr entry is set to 0, so the mask reads as empty: an attention call made
+ * on it anyway loads no tile, and its outputs carry no meaning. Host-visible
+ * argument errors are returned at once and nothing is launched.
  */
 kvs_status kvs_build_tile_mask_async(const kvs_evict_range *ev, int32_t n_ev, int32_t B, int32_t N,
                                      kvs_tile_mask *m, int64_t *dev_sizes, void *ws, size_t ws_bytes,
