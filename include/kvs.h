@@ -126,7 +126,8 @@ kvs_status kvs_build_tile_mask(const kvs_evict_range *ev, int32_t n_ev, int32_t 
                                kvs_stream_t stream);
 
 /*
- * The same compilation without the host round trip, for a training loop that
+ * The same compilation ([T] trainer replay; [P] Fig. 2(A)) without the host
+ * round trip, for a training loop that
  * keeps the mask buffers from step to step: nothing is read back and `stream`
  * is never synchronised, so the call neither stalls the host nor waits behind
  * other device-to-host copies.
