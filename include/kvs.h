@@ -127,10 +127,9 @@ kvs_status kvs_build_tile_mask(const kvs_evict_range *ev, int32_t n_ev, int32_t 
 
 /*
  * The same compilation ([T] trainer replay; [P] Fig. 2(A)) without the host
- * round trip, for a training loop that
- * keeps the mask buffers from step to step: nothing is read back and `stream`
- * is never synchronised, so the call neither stalls the host nor waits behind
- * other device-to-host copies.
+ * round trip, for a training loop that keeps the mask buffers from step to
+ * step: nothing is read back and `stream` is never synchronised, so the call
+ * neither stalls the host nor waits behind other device-to-host copies.
  *   m          as above, with every list pointer set (bits may be NULL only
  *              when partial_cap == 0) and nnz_cap / partial_cap the capacity
  *              of the buffers, e.g. from a counting call on the same log or a
