@@ -7,7 +7,8 @@ budget 32768, whole unpadded turns of 64..4096 tokens evicted at arbitrary
 offsets, 15 events per trace):
 
   training side   event log -> tile mask (kill times, classes, row/col lists,
-                  partial bits); logical RoPE of q and k; eviction-masked
+                  partial bits), recompiled each step into the buffers counted
+                  at set-up with no host round trip; logical RoPE of q and k; eviction-masked
                   attention forward; backward (prep, dK/dV, dQ kernels); inverse
                   RoPE of dq and dk
   generation side block-table compaction at each trace's last event; RoPE of the
