@@ -324,6 +324,12 @@ __global__ void __launch_bounds__(D)
         const int64_t slot = (per_chunk ? dec_cta_of(cs + i, tc, n_cta) : c_first + i) + u;
         return partials + (slot * G + g) * (D + 2);
     };
+    // this thread's dimension of the first pieces, loaded before (and so overlapping)
+    // the two reductions that give the pieces' weights
+    constexpr int kPf = 32;
+    float pv[kPf];
+#pragma unroll
+    for (int i = 0; i < kPf; ++i) pv[i] = i < n_it ? row(i)[e] : 0.f;
     float mloc = -INFINITY;
     for (int i = e; i < n_it; i += D) mloc = fmaxf(mloc, row(i)[D]);
     const float M = block_reduce<D>(mloc, true, s_red);
@@ -337,8 +343,11 @@ __global__ void __launch_bounds__(D)
     }
     const float L = block_reduce<D>(lloc, false, s_red);  // its barriers also publish s_w
     float A = 0.f;
+#pragma unroll
+    for (int i = 0; i < kPf; ++i)
+        if (i < n_it) A += pv[i] * s_w[i];
 #pragma unroll 8
-    for (int i = 0; i < n_it; ++i) A += row(i)[e] * s_w[i];
+    for (int i = kPf; i < n_it; ++i) A += row(i)[e] * s_w[i];
     store_out(o, oi, L > 0.f ? A / L : 0.f);
 }
 
